@@ -1,0 +1,215 @@
+"""fp64 CPU oracle for absorbed MLA decode -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may
+import this package. The product path (``head_latent_attention_split_b200``) never
+does, and the two share no code: the oracle is ``mla_oracle.c`` (plain C, fp64,
+OpenMP over heads) plus the small ctypes wrapper below.
+
+What it computes is stated in ``mla_oracle.c``: the absorbed MLA decode score of
+"TransMLA: Multi-Head Latent Attention Is All You Need" (sec. 3.4.5) with the
+decoupled RoPE term of the TPLA page (sec. 3.4, "The RoPE handling"), a two-pass
+fp64 softmax, and the latent itself as the value.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(worked examples of the "TransMLA & Sparse Latent Attention" lesson, the
+absorbed == explicit identity, GQA == GQA-as-MLA, closed forms, a 50-digit mpmath
+brute force, and library decoders for bf16 / e4m3).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mla_oracle.c")
+_LIB = os.path.join(_HERE, "libmla_oracle.so")
+
+F32, BF16, E4M3, F64 = 0, 1, 2, 3
+
+ERRORS = {0: "ok", 1: "invalid argument", 2: "block id out of range", 3: "seq_len out of range",
+          4: "out of memory"}
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("Sq", ctypes.c_int32), ("H", ctypes.c_int32),
+        ("r", ctypes.c_int32), ("d_r", ctypes.c_int32),
+        ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
+        ("max_blocks_per_seq", ctypes.c_int32),
+        ("q_dtype", ctypes.c_int32), ("cache_dtype", ctypes.c_int32),
+        ("causal", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_double),
+        ("q_lat", ctypes.c_void_p), ("q_rope", ctypes.c_void_p), ("kv_cache", ctypes.c_void_p),
+        ("k_rope_cache", ctypes.c_void_p), ("kv_scale", ctypes.c_void_p),
+        ("block_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+    ]
+
+
+def build(force: bool = False) -> str:
+    """Compile mla_oracle.c into libmla_oracle.so (gcc, -O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                               "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P = ctypes.POINTER(Problem)
+        dp = ctypes.POINTER(ctypes.c_double)
+        L.mla_oracle_decode.argtypes = [P, dp, dp, ctypes.c_int]
+        L.mla_oracle_decode_window.argtypes = [P, ctypes.c_void_p, ctypes.c_void_p, dp, dp, ctypes.c_int]
+        L.mla_oracle_decode_rows.argtypes = [P, ctypes.c_int, ctypes.c_void_p, dp, dp, ctypes.c_int]
+        L.mla_oracle_merge.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, dp, dp, dp, dp]
+        L.mla_oracle_merge.restype = None
+        L.mla_oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        L.mla_oracle_bf16_to_double.restype = ctypes.c_double
+        L.mla_oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        L.mla_oracle_e4m3_to_double.restype = ctypes.c_double
+        _lib = L
+    return _lib
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.float32:
+        return F32
+    if a.dtype == np.uint16:
+        return BF16
+    if a.dtype == np.float64:
+        return F64
+    if a.dtype == np.uint8:
+        return E4M3
+    raise TypeError(f"unsupported oracle input dtype {a.dtype}")
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+class _Bound:
+    """Keeps the numpy inputs alive while the C problem struct points at them."""
+
+    def __init__(self, q_lat, q_rope, kv_cache, block_table, seq_lens, softmax_scale, causal,
+                 k_rope_cache=None, kv_scale=None, block_size=64):
+        self.arrays = [np.ascontiguousarray(x) if x is not None else None
+                       for x in (q_lat, q_rope, kv_cache, k_rope_cache, kv_scale, block_table, seq_lens)]
+        q_lat, q_rope, kv_cache, k_rope_cache, kv_scale, block_table, seq_lens = self.arrays
+        block_table = block_table.astype(np.int32, copy=False)
+        seq_lens = seq_lens.astype(np.int32, copy=False)
+        self.arrays[5], self.arrays[6] = block_table, seq_lens
+        B, Sq, H, r = q_lat.shape
+        d_r = q_rope.shape[-1]
+        cd = _dtype_code(kv_cache)
+        if cd == E4M3:
+            assert kv_scale is not None and kv_scale.dtype == np.float32
+            assert d_r == 0 or (k_rope_cache is not None and k_rope_cache.dtype == np.uint16)
+        qd = _dtype_code(q_lat)
+        assert _dtype_code(q_rope) == qd or q_rope.size == 0
+        self.shape = (B, Sq, H, r, d_r)
+        self.p = Problem(B=B, Sq=Sq, H=H, r=r, d_r=d_r, block_size=block_size,
+                         num_blocks=kv_cache.shape[0], max_blocks_per_seq=block_table.shape[1],
+                         q_dtype=qd, cache_dtype=cd, causal=int(bool(causal)), reserved=0,
+                         softmax_scale=float(softmax_scale),
+                         q_lat=_ptr(q_lat), q_rope=_ptr(q_rope), kv_cache=_ptr(kv_cache),
+                         k_rope_cache=_ptr(k_rope_cache), kv_scale=_ptr(kv_scale),
+                         block_table=_ptr(block_table), seq_lens=_ptr(seq_lens))
+
+
+def _check(rc):
+    if rc != 0:
+        raise RuntimeError(f"oracle error {rc}: {ERRORS.get(rc, '?')}")
+
+
+def _dp(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def decode(q_lat, q_rope, kv_cache, block_table, seq_lens, softmax_scale, causal=False,
+           k_rope_cache=None, kv_scale=None, block_size=64, tok_begin=None, tok_end=None,
+           nthreads=0):
+    """Absorbed MLA decode in fp64. Returns (out [B,Sq,H,r] f64, lse [B,Sq,H] f64).
+
+    Inputs are numpy arrays in their storage format: float32 / float64, uint16 bf16
+    patterns, or uint8 e4m3 codes (cache only, with k_rope_cache bf16 + kv_scale f32).
+    tok_begin / tok_end (int64 [B]) restrict each sequence to a token window.
+    """
+    bd = _Bound(q_lat, q_rope, kv_cache, block_table, seq_lens, softmax_scale, causal,
+                k_rope_cache, kv_scale, block_size)
+    B, Sq, H, r, _ = bd.shape
+    out = np.zeros((B, Sq, H, r), dtype=np.float64)
+    lse = np.zeros((B, Sq, H), dtype=np.float64)
+    if tok_begin is None and tok_end is None:
+        rc = lib().mla_oracle_decode(ctypes.byref(bd.p), _dp(out), _dp(lse), nthreads)
+    else:
+        tb = np.ascontiguousarray(tok_begin, dtype=np.int64) if tok_begin is not None else None
+        te = np.ascontiguousarray(tok_end, dtype=np.int64) if tok_end is not None else None
+        rc = lib().mla_oracle_decode_window(ctypes.byref(bd.p), _ptr(tb), _ptr(te), _dp(out),
+                                            _dp(lse), nthreads)
+    _check(rc)
+    return out, lse
+
+
+def decode_rows(rows, q_lat, q_rope, kv_cache, block_table, seq_lens, softmax_scale, causal=False,
+                k_rope_cache=None, kv_scale=None, block_size=64, nthreads=0):
+    """fp64 decode of selected (b, s, h) rows only. Returns (out [n, r], lse [n])."""
+    bd = _Bound(q_lat, q_rope, kv_cache, block_table, seq_lens, softmax_scale, causal,
+                k_rope_cache, kv_scale, block_size)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+    n = rows.shape[0]
+    r = bd.shape[3]
+    out = np.zeros((n, r), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    _check(lib().mla_oracle_decode_rows(ctypes.byref(bd.p), n, rows.ctypes.data, _dp(out), _dp(lse),
+                                        nthreads))
+    return out, lse
+
+
+def merge(o_parts, lse_parts):
+    """Log-sum-exp merge of partials over disjoint token windows.
+
+    o_parts [P, ..., r], lse_parts [P, ...] -> (out [..., r], lse [...]).
+    """
+    o_parts = np.ascontiguousarray(o_parts, dtype=np.float64)
+    lse_parts = np.ascontiguousarray(lse_parts, dtype=np.float64)
+    P = o_parts.shape[0]
+    r = o_parts.shape[-1]
+    rest = lse_parts.shape[1:]
+    n_rows = int(np.prod(rest)) if rest else 1
+    out = np.zeros(rest + (r,), dtype=np.float64)
+    lse = np.zeros(rest, dtype=np.float64)
+    lib().mla_oracle_merge(P, n_rows, r, _dp(o_parts), _dp(lse_parts), _dp(out), _dp(lse))
+    return out, lse
+
+
+def bf16_to_double(bits: int) -> float:
+    return lib().mla_oracle_bf16_to_double(int(bits))
+
+
+def e4m3_to_double(code: int) -> float:
+    return lib().mla_oracle_e4m3_to_double(int(code))
+
+
+def decode_inputs(inp: dict, nthreads=0, **kw):
+    """Convenience: run ``decode`` on a dict produced by ``workloads.make_inputs``."""
+    w = inp["workload"]
+    return decode(inp["q_lat"], inp["q_rope"], inp["kv_cache"], inp["block_table"], inp["seq_lens"],
+                  w.scale, w.causal, inp.get("k_rope_cache"), inp.get("kv_scale"), w.block_size,
+                  nthreads=nthreads, **kw)
+
+
+def decode_rows_inputs(inp: dict, rows, nthreads=0):
+    w = inp["workload"]
+    return decode_rows(rows, inp["q_lat"], inp["q_rope"], inp["kv_cache"], inp["block_table"],
+                       inp["seq_lens"], w.scale, w.causal, inp.get("k_rope_cache"),
+                       inp.get("kv_scale"), w.block_size, nthreads=nthreads)
