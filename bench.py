@@ -1,0 +1,360 @@
+#!/usr/bin/env python
+"""Benchmark of one absorbed-MLA decode step on B200.
+
+A step = one mla_decode call (split plan + decode kernel + log-sum-exp combine) over the
+whole batch of the chosen workload (default: the DeepSeek-V3-shaped decode, B=64,
+H=128, r=512, d_r=64, 32768-token context, bf16 paged cache). Inputs are seeded
+synthetic data (workloads.py) resident in HBM before timing; the 2.4 GB cache is far
+larger than L2, and workloads whose cache is not are flushed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line on rank 0. `value` is the latent-cache read rate (TB/s of
+attended cache bytes, summed over ranks, over the max-over-ranks device time); TFLOP/s
+and steps/s ride along. With N > 1 (torchrun) every rank runs an independent replica
+(the decode has no cross-GPU exchange). `--impl reference` times the fp64 CPU oracle on
+the host instead, on one sequence per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "MLA decode latent-cache TB/s, TFLOP/s, steps/s; % of roofline at 1 B200"
+FLOP_PER_PAIR = None   # set from the workload: 2 (r + d_r) + 2 r per (query row, head, token)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="deepseek_v3", choices=list(W.BY_NAME))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tcgen05"])
+    ap.add_argument("--num-workers", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained"), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def work_model(inp):
+    """Algorithmic bytes and FLOPs of one step ('Algorithmic work')."""
+    w = inp["workload"]
+    lens = inp["seq_lens"].astype(np.int64)
+    tok = int(lens.sum())
+    per_tok = W.cache_bytes_per_token(w.r, w.d_r, w.cache_dtype)
+    qsz = 4 if w.q_dtype == W.F32 else 2
+    osz = 4 if w.out_dtype == W.F32 else 2
+    rows = w.B * w.Sq * w.H
+    cache_bytes = tok * per_tok
+    io_bytes = rows * (w.r + w.d_r) * qsz + rows * w.r * osz + rows * 4
+    pairs = W.attended_pairs(w, lens)
+    flops = pairs * (2 * (w.r + w.d_r) + 2 * w.r)
+    return dict(tokens=tok, cache_bytes=cache_bytes, io_bytes=io_bytes, bytes=cache_bytes + io_bytes,
+                flops=flops, pairs=pairs)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms in the background."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_id), f"--query-gpu=timestamp,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        rows = []
+        for line in open(self.file.name):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        inside = [r for r in rows if self.t0 - 1 <= r[0] <= self.t1 + 1] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return dict(sm_mhz=statistics.median(r[1] for r in inside), sm_max_mhz=max(r[2] for r in inside),
+                    reasons=reasons, samples=len(inside))
+
+
+def cpu_oracle_rate(inp, seconds, seqs_per_step=None):
+    """Time the fp64 oracle on whole sequences (all heads) until `seconds` elapse."""
+    import oracle
+    w = inp["workload"]
+    per_tok = W.cache_bytes_per_token(w.r, w.d_r, w.cache_dtype)
+    cores = os.cpu_count() or 1
+    done_bytes, elapsed, nseq = 0, 0.0, 0
+    b = 0
+    while (seqs_per_step is None and elapsed < seconds and b < w.B) or (seqs_per_step and nseq < seqs_per_step):
+        sl = slice(b, b + 1)
+        t0 = time.perf_counter()
+        oracle.decode(inp["q_lat"][sl], inp["q_rope"][sl], inp["kv_cache"], inp["block_table"][sl],
+                      inp["seq_lens"][sl], w.scale, w.causal, inp.get("k_rope_cache"), inp.get("kv_scale"),
+                      w.block_size, nthreads=cores)
+        elapsed += time.perf_counter() - t0
+        done_bytes += int(inp["seq_lens"][b]) * per_tok
+        nseq += 1
+        b = (b + 1) % w.B
+    return dict(value=done_bytes / elapsed / 1e12, unit="TB/s", cores=cores, kind="oracle",
+                sample=f"{nseq} of {w.B} sequences (all {w.Sq * w.H} query rows each, full context), "
+                       f"{elapsed:.1f} s of fp64 CPU work"), elapsed
+
+
+def reference_arm(args, rank):
+    if rank != 0:
+        return
+    wl = W.BY_NAME[args.workload]
+    inp = W.make_inputs(wl)
+    per_tok = W.cache_bytes_per_token(wl.r, wl.d_r, wl.cache_dtype)
+    for i in range(args.warmup):
+        cpu_oracle_rate(inp, 0, seqs_per_step=1)
+    tot_t, tot_bytes, tot_flops = 0.0, 0, 0
+    for i in range(args.steps):
+        b = i % wl.B
+        sub = dict(inp, q_lat=inp["q_lat"][b:b + 1], q_rope=inp["q_rope"][b:b + 1],
+                   block_table=inp["block_table"][b:b + 1], seq_lens=inp["seq_lens"][b:b + 1])
+        import oracle
+        t0 = time.perf_counter()
+        oracle.decode_inputs(sub, nthreads=os.cpu_count() or 1)
+        tot_t += time.perf_counter() - t0
+        L = int(inp["seq_lens"][b])
+        tot_bytes += L * per_tok
+        tot_flops += W.attended_pairs(wl.with_(B=1, seq_lens=(L,)), np.array([L])) * (4 * wl.r + 2 * wl.d_r)
+    value = tot_bytes / tot_t / 1e12
+    cores = os.cpu_count() or 1
+    line = dict(metric=METRIC, value=value, unit="TB/s", impl="reference", n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=1e3 * tot_t / args.steps, higher_is_better=True, scaling="weak",
+                vs_baseline=None, dtype="f64", data="synthetic",
+                config=dict(workload=wl.name, B=wl.B, Sq=wl.Sq, H=wl.H, r=wl.r, d_r=wl.d_r,
+                            cache=W.DTYPE_NAMES[wl.cache_dtype], seq_lens=str(wl.seq_lens)[:40],
+                            step="one sequence (all heads) of the workload per step"),
+                tflops=tot_flops / tot_t / 1e12,
+                cpu_baseline=dict(value=value, unit="TB/s", cores=cores, kind="oracle",
+                                  sample=f"one of {wl.B} sequences per step, all {wl.Sq * wl.H} query rows"),
+                e2e=dict(value=value, unit="TB/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import datetime
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+
+    import head_latent_attention_split_b200 as mla
+    wl = W.BY_NAME[args.workload]
+    inp = W.make_inputs(wl, threads=max(1, (os.cpu_count() or 1) // world))
+    t = W.to_torch(inp, f"cuda:{local}")
+    p = mla.params_for(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], wl.scale, wl.causal,
+                       num_workers=args.num_workers, kernel=args.kernel)
+    kernel, workers = mla.resolve(p)
+    ws = torch.empty(max(1, mla.workspace_size(p)), dtype=torch.uint8, device=t["q_lat"].device)
+    out = torch.empty(t["q_lat"].shape, dtype=torch.bfloat16 if wl.out_dtype == W.BF16 else torch.float32,
+                      device=t["q_lat"].device)
+    lse = torch.empty(t["q_lat"].shape[:3], dtype=torch.float32, device=t["q_lat"].device)
+    model = work_model(inp)
+    props = torch.cuda.get_device_properties(local)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+    resident = sum(x.numel() * x.element_size() for k, x in t.items() if k != "workload" and x is not None)
+    flush = model["cache_bytes"] < 8 * l2
+    flush_buf = torch.empty(2 * l2 // 4 + 1, dtype=torch.float32, device=out.device) if flush else None
+
+    def step(ev=None):
+        if ev is None:
+            mla.mla_decode(p, t["q_lat"], t["q_rope"], t["kv_cache"], t["k_rope_cache"], t["kv_scale"],
+                           t["block_table"], t["seq_lens"], out, lse, ws)
+        else:
+            mla.mla_decode_timed(p, t["q_lat"], t["q_rope"], t["kv_cache"], t["k_rope_cache"], t["kv_scale"],
+                                 t["block_table"], t["seq_lens"], out, lse, ws, ev)
+
+    for _ in range(max(3, args.warmup)):
+        if flush:
+            flush_buf.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    st = mla.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {mla.status_string(st)}")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for e in evs:          # create the underlying CUDA events
+        for x in e:
+            x.record()
+    torch.cuda.synchronize()
+    gpu_id = getattr(props, "uuid", None)
+    sampler = ClockSampler(f"GPU-{gpu_id}" if gpu_id is not None else local)
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.mark_start()
+    for i in range(K):
+        if flush:
+            flush_buf.fill_(1.0)
+        step(evs[i])
+    torch.cuda.synchronize()
+    sampler.mark_end()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    dec_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    comb_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms = sum(step_ms)
+    tot = torch.tensor([total_ms], dtype=torch.float64, device=out.device)
+    if world > 1:
+        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
+    total_ms = float(tot.item())
+    st = mla.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {mla.status_string(st)}")
+
+    # end-to-end through the host-buffer entry point: per-step inputs copied from pinned
+    # host memory, result copied back, all inside the timed region
+    E = args.e2e_steps if args.e2e_steps is not None else max(1, min(K, 50))
+    pin = lambda x: x.cpu().pin_memory()
+    hq, hqr, hbt, hsl = pin(t["q_lat"]), pin(t["q_rope"]), pin(t["block_table"]), pin(t["seq_lens"])
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    hlse = torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
+    hws = torch.empty(mla.host_io_workspace_size(p), dtype=torch.uint8, device=out.device)
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hqr, hbt, hsl))
+    d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
+    e2e_ms = 0.0
+    for i in range(E + 2):
+        if flush:
+            flush_buf.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        mla.mla_decode_host_io(p, hq, hqr, t["kv_cache"], t["k_rope_cache"], t["kv_scale"], hbt, hsl, hout, hlse,
+                               hws)
+        b.record()
+        b.synchronize()
+        if i >= 2:
+            e2e_ms += a.elapsed_time(b)
+    e2e = torch.tensor([e2e_ms], dtype=torch.float64, device=out.device)
+    if world > 1:
+        dist.all_reduce(e2e, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e.item())
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu, _ = cpu_oracle_rate(inp, args.cpu_seconds)
+
+    if rank == 0:
+        peaks = load_peaks()
+        sec = total_ms / 1e3
+        value = world * K * model["cache_bytes"] / sec / 1e12
+        dec_s = statistics.mean(dec_ms) / 1e3
+        t_hbm = model["bytes"] / (peaks["hbm_gbs"] * 1e9)
+        t_tc = model["flops"] / (peaks["bf16_tflops"] * 1e12)
+        bound = "hbm" if t_hbm >= t_tc else "tensor"
+        if bound == "hbm":
+            achieved, peak, unit = model["bytes"] / dec_s / 1e9, peaks["hbm_gbs"], "GB/s"
+        else:
+            achieved, peak, unit = model["flops"] / dec_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        line = dict(
+            metric=METRIC, value=value, unit="TB/s", n_gpus=world, steps=K, warmup=args.warmup,
+            ms_per_step=total_ms / K, higher_is_better=True, scaling="weak", vs_baseline=None,
+            dtype=W.DTYPE_NAMES[wl.cache_dtype] if wl.cache_dtype != W.E4M3 else "e4m3+bf16",
+            data="synthetic",
+            config=dict(workload=wl.name, B=wl.B, Sq=wl.Sq, H=wl.H, r=wl.r, d_r=wl.d_r, block_size=wl.block_size,
+                        context=str(wl.seq_lens) if isinstance(wl.seq_lens, str) else int(max(wl.seq_lens)),
+                        cache=W.DTYPE_NAMES[wl.cache_dtype], kernel=kernel, workers=workers,
+                        parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                        l2=("flushed between steps (2x L2 buffer write)" if flush else
+                            f"inputs larger than L2 ({model['cache_bytes'] / 1e9:.2f} GB cache per step)"),
+                        resident_bytes=resident),
+            tflops=world * K * model["flops"] / sec / 1e12,
+            steps_per_s=K / sec,
+            tokens_per_s=world * K * wl.B * wl.Sq / sec,
+            roofline=dict(bound=bound, achieved=achieved, peak=peak, unit=unit, frac=achieved / peak,
+                          traffic=None),
+            roofline_detail=dict(
+                kernel=f"decode ({kernel})", decode_ms=1e3 * dec_s, combine_ms=statistics.mean(comb_ms),
+                algorithmic_bytes=model["bytes"], algorithmic_flops=model["flops"],
+                hbm_gbs_achieved=model["bytes"] / dec_s / 1e9, tflops_achieved=model["flops"] / dec_s / 1e12,
+                hbm_frac=model["bytes"] / dec_s / 1e9 / peaks["hbm_gbs"],
+                tensor_frac=model["flops"] / dec_s / 1e12 / peaks["bf16_tflops"],
+                roofline_us=1e6 * max(t_hbm, t_tc), step_frac=max(t_hbm, t_tc) / (total_ms / K / 1e3),
+                peaks=peaks),
+            cpu_baseline=cpu,
+            e2e=dict(value=world * E * model["cache_bytes"] / (e2e_ms / 1e3) / 1e12, unit="TB/s",
+                     h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms / E),
+            gpu_launches=2 * K,
+            clocks=clocks,
+        )
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,12 @@
+"""Absorbed multi-head latent attention (MLA) decode for B200 (sm_100a).
+
+One decode step over a paged, compressed latent KV cache: every query head scores its
+absorbed query against each cached token's latent c_t (plus the decoupled RoPE key)
+and sums the latents back with the softmax weights, so one latent tile serves as both
+key and value. The kernels live in libmla_decode.so (C ABI: include/mla_decode.h);
+this package is a thin binding over it.
+"""
+from .binding import (BF16, E4M3, F32, KERNELS, MlaError, Params, abi_version, device_status,  # noqa: F401
+                      host_io_workspace_size, make_params, mla_decode, mla_decode_host_io, mla_decode_timed, plan_host,
+                      plan_probe, resolve, status_string, workspace_size)
+from .api import decode, decode_host_io, params_for  # noqa: F401

@@ -1,0 +1,73 @@
+"""torch-tensor front end of the C ABI: shape/dtype inference and output allocation."""
+from __future__ import annotations
+
+from . import binding as _b
+
+
+def _dtype_code(t, what):
+    import torch
+    if t.dtype == torch.float32:
+        return _b.F32
+    if t.dtype == torch.bfloat16:
+        return _b.BF16
+    if t.dtype in (torch.uint8, getattr(torch, "float8_e4m3fn", None)):
+        return _b.E4M3
+    raise TypeError(f"{what}: unsupported dtype {t.dtype}")
+
+
+def params_for(q_lat, q_rope, kv_cache, block_table, softmax_scale, causal=False, out_dtype=None,
+               num_workers=0, kernel="auto") -> _b.Params:
+    """Build mla_decode_params_t from tensor shapes.
+
+    q_lat [B, Sq, H, r], q_rope [B, Sq, H, d_r], kv_cache [num_blocks, block_size, r + d_r]
+    (f32 / bf16) or e4m3 codes [num_blocks, block_size, r], block_table [B, max_blocks].
+    """
+    B, Sq, H, r = q_lat.shape
+    d_r = q_rope.shape[-1] if q_rope is not None else 0
+    qd = _dtype_code(q_lat, "q_lat")
+    cd = _dtype_code(kv_cache, "kv_cache")
+    od = qd if out_dtype is None else out_dtype
+    nb, bs = kv_cache.shape[0], kv_cache.shape[1]
+    return _b.make_params(B, Sq, H, r, d_r, bs, nb, block_table.shape[1], qd, cd, od, causal, softmax_scale,
+                          num_workers, kernel)
+
+
+def decode(q_lat, q_rope, kv_cache, block_table, seq_lens, softmax_scale, causal=False, k_rope_cache=None,
+           kv_scale=None, out=None, lse=None, workspace=None, out_dtype=None, num_workers=0, kernel="auto",
+           stream=None):
+    """One MLA decode step on the current CUDA device. Returns (out, lse).
+
+    out [B, Sq, H, r] (dtype of q unless out_dtype), lse [B, Sq, H] float32 (natural log).
+    """
+    import torch
+    p = params_for(q_lat, q_rope, kv_cache, block_table, softmax_scale, causal, out_dtype, num_workers, kernel)
+    dev = q_lat.device
+    if out is None:
+        od = {_b.F32: torch.float32, _b.BF16: torch.bfloat16}[p.out_dtype]
+        out = torch.empty(q_lat.shape, dtype=od, device=dev)
+    if lse is None:
+        lse = torch.empty(q_lat.shape[:3], dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(_b.workspace_size(p), 1), dtype=torch.uint8, device=dev)
+    _b.mla_decode(p, q_lat, q_rope, kv_cache, k_rope_cache, kv_scale, block_table, seq_lens, out, lse, workspace,
+                  stream=stream)
+    return out, lse
+
+
+def decode_host_io(q_lat_host, q_rope_host, kv_cache, block_table_host, seq_lens_host, softmax_scale,
+                   causal=False, k_rope_cache=None, kv_scale=None, out_host=None, lse_host=None, workspace=None,
+                   out_dtype=None, num_workers=0, kernel="auto", stream=None):
+    """Decode step with per-step tensors in pinned host memory (see mla_decode_host_io)."""
+    import torch
+    p = params_for(q_lat_host, q_rope_host, kv_cache, block_table_host, softmax_scale, causal, out_dtype,
+                   num_workers, kernel)
+    if out_host is None:
+        od = {_b.F32: torch.float32, _b.BF16: torch.bfloat16}[p.out_dtype]
+        out_host = torch.empty(q_lat_host.shape, dtype=od, pin_memory=True)
+    if lse_host is None:
+        lse_host = torch.empty(q_lat_host.shape[:3], dtype=torch.float32, pin_memory=True)
+    if workspace is None:
+        workspace = torch.empty(_b.host_io_workspace_size(p), dtype=torch.uint8, device=kv_cache.device)
+    _b.mla_decode_host_io(p, q_lat_host, q_rope_host, kv_cache, k_rope_cache, kv_scale, block_table_host,
+                          seq_lens_host, out_host, lse_host, workspace, stream=stream)
+    return out_host, lse_host

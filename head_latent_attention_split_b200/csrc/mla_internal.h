@@ -1,0 +1,74 @@
+// Internal interface between the C-ABI host layer (mla_api.cu) and the kernel
+// translation units. Not installed; the public interface is include/mla_decode.h.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace mla {
+
+enum : int { kF32 = 0, kBF16 = 1, kE4M3 = 2 };
+
+// Everything a decode / combine / probe kernel needs, by value.
+struct DecodeArgs {
+  int B, Sq, H, r, d_r;
+  int bs;              // block_size (tokens per cache block)
+  int num_blocks;
+  int max_blocks;      // block_table row stride
+  int q_dtype, cache_dtype, out_dtype;
+  int causal;
+  int rows;            // Sq * H query rows per sequence
+  int W;               // workers sharing the flat block list
+  float scale;         // softmax scale
+  float scale_log2;    // softmax scale * log2(e)
+  const void* q_lat;
+  const void* q_rope;
+  const void* cache;           // F32/BF16: [nb, bs, r + d_r]; E4M3: codes [nb, bs, r]
+  const uint16_t* k_rope;      // E4M3 only: bf16 [nb, bs, d_r]
+  const float* kv_scale;       // E4M3 only: [nb, bs]
+  const int32_t* block_table;  // [B, max_blocks]
+  const int32_t* seq_lens;     // [B]
+  void* out;                   // [B, Sq, H, r] out_dtype
+  float* lse;                  // [B, Sq, H]
+  // workspace
+  int32_t* meta;               // [B, 2]: first worker, number of splits
+  float* lse_part;             // [slots, rows]
+  float* o_part;               // [slots, rows, r] (normalised partial outputs)
+  int* status;                 // sticky device status word
+};
+
+// Workspace regions; every offset is 256-byte aligned.
+struct WorkspaceLayout {
+  size_t meta_off, lse_off, o_off, total;
+  int64_t slots;
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline WorkspaceLayout workspace_layout(int B, int W, int rows, int r) {
+  WorkspaceLayout L;
+  // worker w's part of sequence b uses slot w + b (unique: workers own increasing,
+  // contiguous block ranges of the batch-ordered block list)
+  L.slots = (B > 0 && W > 0) ? (int64_t)W + B - 1 : 0;
+  L.meta_off = 0;
+  L.lse_off = align_up(sizeof(int32_t) * 2 * (size_t)B, 256);
+  L.o_off = L.lse_off + align_up(sizeof(float) * (size_t)L.slots * rows, 256);
+  L.total = L.o_off + align_up(sizeof(float) * (size_t)L.slots * rows * r, 256);
+  return L;
+}
+
+// SIMT (CUDA-core, fp32) decode: any r <= kSimtMaxR, r + d_r <= kSimtMaxD.
+constexpr int kSimtMaxR = 1024;
+constexpr int kSimtMaxD = 1280;
+cudaError_t launch_simt_decode(const DecodeArgs& a, cudaStream_t s);
+
+// Log-sum-exp merge of split partials (and the fill of empty sequences).
+cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
+
+// Plan probe for tests.
+cudaError_t launch_plan_probe(const DecodeArgs& a, int32_t* token_slot, int32_t* token_worker,
+                              cudaStream_t s);
+
+}  // namespace mla

@@ -1,0 +1,191 @@
+/*
+ * mla_decode.h -- C ABI of the B200 (sm_100a) absorbed multi-head latent attention
+ * (MLA) decode library, libmla_decode.so.
+ *
+ * The operation. One decode step of one attention layer for a batch of sequences
+ * whose keys and values live in a shared compressed latent cache:
+ *
+ *   for every sequence b, query position s < Sq, head h:
+ *     sigma_t = softmax_scale * ( q_lat[b,s,h,:] . c_t  +  q_rope[b,s,h,:] . kR_t )
+ *     lse[b,s,h]   = log sum_t exp(sigma_t)                      (natural log)
+ *     out[b,s,h,:] = sum_t exp(sigma_t - lse[b,s,h]) * c_t
+ *
+ *   c_t (kv_rank = r values) is token t's cached latent and serves as both the key
+ *   content and the value; kR_t (rope_dim = d_r values) is its decoupled RoPE key,
+ *   shared by all heads. q_lat is the absorbed query (W^UK folded into the query
+ *   projection) and q_rope the RoPE part of the query.
+ *   Sources: "TransMLA: Multi-Head Latent Attention Is All You Need" (paper-graph
+ *   summary), sec. 3.4.5 "The full MLA structure after conversion" (absorbed query
+ *   [(W^UK_i)^T q; q^R] against the cached [c^KV; k^R]); TPLA paper-graph summary,
+ *   sec. 3.4, eq. 5 (softmax(Q c^T) c: the latent is the value) and "The RoPE
+ *   handling" (score = (Q c^T + q^PE k^PE^T) / sqrt(d_h + d_r)). The caller passes the
+ *   scale, so any of the pages' temperature conventions can be used.
+ *
+ *   Attended tokens: with causal == 0 every query row sees tokens [0, seq_lens[b]).
+ *   With causal != 0 the Sq queries are the last Sq tokens of the sequence and query
+ *   s sees tokens [0, seq_lens[b] - Sq + 1 + s). A row that sees no token gets
+ *   out = 0 and lse = -inf.
+ *
+ * Cache layout (paged). Token t of sequence b is slot t % block_size of physical
+ * block block_table[b * max_blocks_per_seq + t / block_size].
+ *   cache_dtype F32 / BF16: kv_cache = [num_blocks, block_size, r + d_r], latent then
+ *     RoPE key, row-major. k_rope_cache and kv_scale must be NULL.
+ *   cache_dtype E4M3 (OCP FP8 e4m3, no infinities): kv_cache = codes
+ *     [num_blocks, block_size, r] (uint8); c_t = decode(code) * kv_scale[slot];
+ *     k_rope_cache = bf16 [num_blocks, block_size, d_r]; kv_scale = f32
+ *     [num_blocks, block_size].
+ *   Slots past a sequence's length in its last block are never read for scores or
+ *   values (they may hold anything, NaN included).
+ *
+ * Other tensors (all contiguous, row-major, device-resident unless stated):
+ *   q_lat  [B, Sq, H, r]   q_dtype        q_rope [B, Sq, H, d_r] q_dtype
+ *   block_table [B, max_blocks_per_seq] int32     seq_lens [B] int32
+ *   out    [B, Sq, H, r]   out_dtype      lse    [B, Sq, H] float32
+ * Supported dtype triples (q, cache, out): (F32, F32, F32), (BF16, BF16, BF16|F32),
+ * (BF16, E4M3, BF16|F32).
+ *
+ * Ownership and threading. The caller owns every buffer, the workspace included;
+ * the library never allocates device memory. Calls are stream-ordered and
+ * asynchronous: they enqueue work on `stream` (a cudaStream_t, NULL = legacy default
+ * stream) on the current device and return. Concurrent calls on different streams
+ * need different workspaces.
+ *
+ * Errors. Argument errors are detected on the host before anything is enqueued and
+ * returned synchronously (nothing is launched). A failed launch returns MLA_ERR_CUDA.
+ * Data-dependent errors found on the device (a block id outside [0, num_blocks), a
+ * seq_len outside [0, max_blocks_per_seq * block_size], a bounded wait that timed
+ * out) do not stop the kernels: the offending block id is replaced by block 0 and the
+ * seq_len clamped, so the results for that sequence are meaningless, and a sticky
+ * per-device status word records the first such error. mla_get_device_status() reads
+ * and clears it. No device code traps.
+ */
+#ifndef MLA_DECODE_H_
+#define MLA_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_DECODE_ABI_VERSION 1
+
+typedef enum { MLA_DTYPE_F32 = 0, MLA_DTYPE_BF16 = 1, MLA_DTYPE_E4M3 = 2 } mla_dtype_t;
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,         /* bad shape, NULL pointer, bad dtype combination */
+  MLA_ERR_UNSUPPORTED = 2,         /* valid request that the chosen kernel cannot run */
+  MLA_ERR_ALIGNMENT = 3,           /* a device pointer is not 16-byte aligned */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 4,
+  MLA_ERR_CUDA = 5,                /* CUDA runtime / launch error */
+  MLA_ERR_BAD_BLOCK_ID = 6,        /* device-detected, sticky */
+  MLA_ERR_BAD_SEQ_LEN = 7,         /* device-detected, sticky */
+  MLA_ERR_TIMEOUT = 8              /* device-detected bounded wait expiry, sticky */
+} mla_status_t;
+
+typedef enum {
+  MLA_KERNEL_AUTO = 0,     /* tensor-core kernel when the shape allows it, else SIMT */
+  MLA_KERNEL_SIMT = 1,     /* fp32 CUDA-core kernel: any r <= 1024, r + d_r <= 1280 */
+  MLA_KERNEL_TCGEN05 = 2   /* tcgen05/TMA kernel: r = 512, d_r = 64, block_size = 64 */
+} mla_kernel_t;
+
+typedef struct {
+  int32_t batch;               /* B >= 0 */
+  int32_t q_len;               /* Sq >= 1 query tokens per sequence */
+  int32_t num_heads;           /* H >= 1 */
+  int32_t kv_rank;             /* r >= 1, latent width */
+  int32_t rope_dim;            /* d_r >= 0, decoupled RoPE key width */
+  int32_t block_size;          /* tokens per cache block */
+  int32_t num_blocks;          /* physical blocks in the cache */
+  int32_t max_blocks_per_seq;  /* row stride of block_table */
+  int32_t q_dtype;             /* mla_dtype_t */
+  int32_t cache_dtype;         /* mla_dtype_t */
+  int32_t out_dtype;           /* mla_dtype_t */
+  int32_t causal;              /* 0 / 1, see above */
+  float softmax_scale;         /* multiplies the summed score; finite */
+  int32_t num_workers;         /* 0 = auto; else the number of KV-range workers */
+  int32_t kernel;              /* mla_kernel_t */
+  int32_t reserved;            /* must be 0 */
+} mla_decode_params_t;
+
+/* Bytes of device workspace mla_decode needs for these parameters (host only; with
+ * num_workers == 0 it queries the current device's SM count). The bound does not
+ * depend on seq_lens. */
+mla_status_t mla_decode_workspace_size(const mla_decode_params_t* params, size_t* bytes);
+
+/* Kernel and worker count a call with these parameters would use (host only). */
+mla_status_t mla_decode_resolve(const mla_decode_params_t* params, int32_t* kernel,
+                                int32_t* num_workers);
+
+/* Enqueue one decode step (see the header comment). All tensor pointers are device
+ * pointers. workspace must hold mla_decode_workspace_size() bytes, 256-byte aligned;
+ * its contents need no initialisation and are clobbered. */
+mla_status_t mla_decode(const mla_decode_params_t* params, const void* q_lat, const void* q_rope,
+                        const void* kv_cache, const void* k_rope_cache, const float* kv_scale,
+                        const int32_t* block_table, const int32_t* seq_lens, void* out, float* lse,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* mla_decode, plus three CUDA events (cudaEvent_t, created by the caller) recorded on
+ * `stream`: events[0] before the decode kernel, events[1] between the decode kernel
+ * and the split-combine kernel, events[2] after the combine. Lets a caller time each
+ * kernel of the step on the launching stream; the work done is identical. */
+mla_status_t mla_decode_timed(const mla_decode_params_t* params, const void* q_lat, const void* q_rope,
+                              const void* kv_cache, const void* k_rope_cache, const float* kv_scale,
+                              const int32_t* block_table, const int32_t* seq_lens, void* out, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream,
+                              void* const* events);
+
+/* Bytes of device workspace mla_decode_host_io needs: device staging for the per-step
+ * inputs and outputs plus mla_decode's own workspace. */
+mla_status_t mla_decode_host_io_workspace_size(const mla_decode_params_t* params, size_t* bytes);
+
+/* One decode step whose per-step tensors are in HOST memory (pinned memory makes the
+ * copies asynchronous): q_lat, q_rope, block_table, seq_lens are copied to the
+ * device, the step runs, out and lse are copied back, all on `stream`. The cache
+ * (kv_cache, k_rope_cache, kv_scale) stays device-resident. The call returns once
+ * the work is enqueued; synchronise the stream before reading out / lse. */
+mla_status_t mla_decode_host_io(const mla_decode_params_t* params, const void* q_lat_host,
+                                const void* q_rope_host, const void* kv_cache,
+                                const void* k_rope_cache, const float* kv_scale,
+                                const int32_t* block_table_host, const int32_t* seq_lens_host,
+                                void* out_host, float* lse_host, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* Split plan on the host, for tests. Work is the flat list of cache blocks of all
+ * sequences in batch order; worker w of W owns blocks [floor(w*T/W), floor((w+1)*T/W))
+ * of the T blocks. Outputs (host arrays): seq_block_begin[B + 1] (prefix of blocks per
+ * sequence), seq_first_worker[B] and seq_num_splits[B] (workers that touch each
+ * sequence; 0 splits for an empty sequence). W comes from mla_decode_resolve. */
+mla_status_t mla_plan_host(const mla_decode_params_t* params, const int32_t* seq_lens_host,
+                           int32_t* seq_block_begin, int32_t* seq_first_worker,
+                           int32_t* seq_num_splits);
+
+/* Device probe of the same plan, for tests: every worker walks its block range with
+ * the device code the decode kernels use and records, for each logical token t of
+ * sequence b, the physical slot it reads (block * block_size + offset) in
+ * token_slot[b * max_blocks_per_seq * block_size + t] and its worker id in
+ * token_worker[...]; unread entries are left untouched. seq_meta[2 * b] and
+ * seq_meta[2 * b + 1] receive the first worker and split count the kernels use.
+ * All pointers are device pointers. */
+mla_status_t mla_plan_probe(const mla_decode_params_t* params, const int32_t* block_table,
+                            const int32_t* seq_lens, int32_t* token_slot, int32_t* token_worker,
+                            int32_t* seq_meta, void* stream);
+
+/* Synchronise `stream`, then read and clear the current device's sticky status word
+ * (MLA_OK or one of the device-detected codes). Returns MLA_ERR_CUDA if the
+ * synchronisation itself failed. */
+mla_status_t mla_get_device_status(void* stream, int32_t* device_status);
+
+/* Static, human-readable name of a status code. */
+const char* mla_status_string(int32_t status);
+
+/* MLA_DECODE_ABI_VERSION of the loaded library. */
+int32_t mla_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H_ */

@@ -1,0 +1,162 @@
+"""CPU-only checks of the C-ABI library: it loads, exports what include/mla_decode.h
+declares, rejects bad arguments before touching the GPU, and plans splits as defined."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla_decode.h")
+
+
+@pytest.fixture(scope="module")
+def m():
+    from head_latent_attention_split_b200 import build as B
+    B.build()
+    import head_latent_attention_split_b200 as mod
+    return mod
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(mla_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("mla_decode", "mla_decode_workspace_size", "mla_get_device_status", "mla_plan_host"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(m):
+    from head_latent_attention_split_b200 import binding
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (mla_\w+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(binding.lib, name)
+    assert set(binding.EXPORTED) <= exported
+    assert m.abi_version() == 1
+
+
+def test_library_has_no_torch_or_libcuda_dependency(m):
+    from head_latent_attention_split_b200 import binding
+    out = subprocess.run(["readelf", "-d", binding.LIB_PATH], capture_output=True, text=True).stdout
+    needed = re.findall(r"\(NEEDED\).*\[(.*)\]", out)
+    assert not any("torch" in n or n.startswith("libcuda.so") or "c10" in n for n in needed), needed
+
+
+def _p(m, **kw):
+    base = dict(B=2, Sq=1, H=4, r=16, d_r=8, block_size=64, num_blocks=2, max_blocks_per_seq=1,
+                q_dtype=0, cache_dtype=0, out_dtype=0, causal=False, softmax_scale=0.2, num_workers=3,
+                kernel="simt")
+    base.update(kw)
+    return m.make_params(**base)
+
+
+FAKE = 1 << 20   # a 256-byte aligned address that is never dereferenced
+
+
+def _call(m, p, **ptrs):
+    from head_latent_attention_split_b200 import binding
+    args = dict(q_lat=FAKE, q_rope=FAKE, kv_cache=FAKE, k_rope_cache=None, kv_scale=None, block_table=FAKE,
+                seq_lens=FAKE, out=FAKE, lse=FAKE, workspace=FAKE, workspace_bytes=1 << 30)
+    args.update(ptrs)
+    return binding.mla_decode(p, stream=0, check=False, **args)
+
+
+@pytest.mark.parametrize("bad", [dict(Sq=0), dict(H=0), dict(r=0), dict(d_r=-1), dict(block_size=0),
+                                 dict(max_blocks_per_seq=0), dict(q_dtype=7), dict(q_dtype=1),
+                                 dict(cache_dtype=2, q_dtype=0), dict(out_dtype=2, q_dtype=1, cache_dtype=1),
+                                 dict(softmax_scale=float("nan")), dict(causal=2), dict(kernel=9),
+                                 dict(num_workers=-1), dict(num_blocks=0)])
+def test_invalid_params_rejected_on_host(m, bad):
+    causal = bad.pop("causal", None)
+    p = _p(m, **bad)
+    if causal is not None:
+        p.causal = causal          # make_params would coerce it to 0/1
+    assert _call(m, p) == 1     # MLA_ERR_INVALID_ARG, nothing launched
+
+
+def test_null_pointers_rejected(m):
+    p = _p(m)
+    for k in ("q_lat", "kv_cache", "block_table", "seq_lens", "out", "lse", "workspace", "q_rope"):
+        assert _call(m, p, **{k: None}) == 1, k
+    # e4m3 needs its rope plane and scales; f32/bf16 must not get them
+    p8 = _p(m, q_dtype=1, cache_dtype=2, out_dtype=1)
+    assert _call(m, p8) == 1
+    assert _call(m, p, kv_scale=FAKE) == 1
+
+
+def test_workspace_and_alignment_checks(m):
+    p = _p(m)
+    need = m.workspace_size(p)
+    assert _call(m, p, workspace_bytes=need - 1) == 4           # MLA_ERR_WORKSPACE_TOO_SMALL
+    assert _call(m, p, workspace=FAKE + 16, workspace_bytes=need) == 3   # MLA_ERR_ALIGNMENT
+    assert _call(m, p, out=FAKE + 2, workspace_bytes=need) == 3
+
+
+def test_unsupported_kernel_requests(m):
+    # the SIMT kernel is limited to r <= 1024, r + d_r <= 1280
+    assert _call(m, _p(m, r=2048)) == 2
+    # the tensor-core kernel needs r = 512, d_r = 64, block 64, bf16 queries
+    assert _call(m, _p(m, kernel="tcgen05")) == 2
+
+
+def test_batch_zero_is_a_noop(m):
+    p = _p(m, B=0)
+    assert _call(m, p, q_lat=None, kv_cache=None) == 0
+
+
+def test_workspace_size_formula(m):
+    p = _p(m, B=5, Sq=2, H=8, r=32, num_workers=7)
+    rows, slots = 2 * 8, 7 + 5 - 1
+    al = lambda x: (x + 255) // 256 * 256
+    assert m.workspace_size(p) == al(5 * 8) + al(slots * rows * 4) + al(slots * rows * 32 * 4)
+
+
+def _plan_by_definition(lens, bs, W):
+    n = [(L + bs - 1) // bs for L in lens]
+    P = np.concatenate([[0], np.cumsum(n)]).astype(np.int64)
+    T = int(P[-1])
+    rng = [(w * T // W, (w + 1) * T // W) for w in range(W)]
+    first, splits = [], []
+    for b in range(len(lens)):
+        touch = [w for w, (s, e) in enumerate(rng) if n[b] and s < e and s < P[b] + n[b] and e > P[b]]
+        first.append(touch[0] if touch else 0)
+        splits.append(len(touch))
+    return P, first, splits, rng
+
+
+@pytest.mark.parametrize("W", [1, 2, 5, 74, 300])
+def test_plan_host_matches_definition(m, W):
+    rng = np.random.default_rng(W)
+    lens = [int(x) for x in rng.integers(0, 3000, size=37)] + [0, 1, 64, 65, 128]
+    B = len(lens)
+    bs = 64
+    p = _p(m, B=B, max_blocks_per_seq=(max(lens) + bs - 1) // bs, num_blocks=10 ** 5, num_workers=W)
+    plan = m.plan_host(p, lens)
+    P, first, splits, ranges = _plan_by_definition(lens, bs, W)
+    np.testing.assert_array_equal(plan["block_begin"], P)
+    np.testing.assert_array_equal(plan["splits"], splits)
+    for b in range(B):
+        if splits[b]:
+            assert plan["first_worker"][b] == first[b]
+    # balance: worker ranges differ by at most one block
+    sizes = [e - s for s, e in ranges]
+    assert max(sizes) - min(sizes) <= 1
+    # workspace slots w + b of all (worker, sequence) pairs are distinct and < W + B - 1
+    slots = [plan["first_worker"][b] + k + b for b in range(B) if splits[b] > 1 for k in range(splits[b])]
+    assert len(slots) == len(set(slots)) and (not slots or max(slots) < W + B - 1)
+
+
+def test_plan_host_rejects_bad_lengths(m):
+    p = _p(m, B=2, max_blocks_per_seq=1)
+    with pytest.raises(Exception):
+        m.plan_host(p, [65, 3])
+    with pytest.raises(Exception):
+        m.plan_host(p, [-1, 3])

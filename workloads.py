@@ -263,3 +263,20 @@ def attended_pairs(w: Workload, lens: np.ndarray) -> int:
             n = int(L) - w.Sq + 1 + s if w.causal else int(L)
             tot += max(0, n)
     return tot * w.H
+
+
+def to_torch(inp: dict, device="cuda") -> dict:
+    """Move the arrays of ``make_inputs`` to torch tensors on ``device`` (bit-exact)."""
+    import torch
+
+    def t(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    out = {k: t(inp[k]) for k in ("q_lat", "q_rope", "kv_cache", "k_rope_cache", "kv_scale", "block_table",
+                                   "seq_lens")}
+    out["workload"] = inp["workload"]
+    return out
