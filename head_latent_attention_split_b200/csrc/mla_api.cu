@@ -330,6 +330,7 @@ mla_status_t mla_plan_host(const mla_decode_params_t* p, const int32_t* seq_lens
     T += (L + p->block_size - 1) / p->block_size;
   }
   if (p->batch >= 0 && seq_block_begin) seq_block_begin[p->batch] = (int32_t)T;
+  const int64_t Wa = (T > 0 && T < W) ? T : W;   // active workers: each owns >= 1 block
   for (int b = 0; b < p->batch; ++b) {
     const int64_t P = seq_block_begin[b], n = seq_block_begin[b + 1] - P;
     if (n == 0) {
@@ -337,8 +338,8 @@ mla_status_t mla_plan_host(const mla_decode_params_t* p, const int32_t* seq_lens
       seq_num_splits[b] = 0;
       continue;
     }
-    // worker containing flat block x: largest w with floor(w T / W) <= x
-    auto owner = [&](int64_t x) { return (int32_t)(((x + 1) * W - 1) / T); };
+    // worker containing flat block x: largest w with floor(w T / Wa) <= x
+    auto owner = [&](int64_t x) { return (int32_t)(((x + 1) * Wa - 1) / T); };
     seq_first_worker[b] = owner(P);
     seq_num_splits[b] = owner(P + n - 1) - owner(P) + 1;
   }

@@ -38,10 +38,11 @@ __device__ __forceinline__ float load_q(const void* p, int dtype, size_t i) {
 // ---------------------------------------------------------------------------- plan
 //
 // The work of one call is the batch-ordered list of every sequence's cache blocks
-// ("tiles"): T = sum_b ceil(L_b / bs). Worker w of W owns tiles
-// [floor(w T / W), floor((w + 1) T / W)). The part of sequence b that worker w owns is
-// one split; the splits of b are numbered from the first worker that touches b, and
-// the split's partial result goes to workspace slot w + b.
+// ("tiles"): T = sum_b ceil(L_b / bs). With W' = min(W, T) active workers, worker
+// w < W' owns tiles [floor(w T / W'), floor((w + 1) T / W')): at least one tile each,
+// so the workers that touch a sequence are consecutive. The part of sequence b that
+// worker w owns is one split; the splits of b are numbered from the first worker that
+// touches b, and the split's partial result goes to workspace slot w + b.
 
 __device__ __forceinline__ int clamp_len(int L, int cap, int* status) {
   if (L < 0 || L > cap) {
@@ -60,6 +61,7 @@ __device__ __forceinline__ int worker_of_tile(long long x, long long T, int W) {
 
 struct WorkerPlan {
   long long T;      // total tiles
+  int W;            // active workers, min(W, T)
   long long start;  // first tile of this worker
   long long end;    // one past its last tile
   long long P0;     // flat index of sequence b0's first tile
@@ -76,8 +78,9 @@ __device__ __forceinline__ WorkerPlan warp_plan(const int32_t* __restrict__ seq_
   for (int o = 16; o > 0; o >>= 1) T += __shfl_xor_sync(0xffffffffu, T, o);
   WorkerPlan p;
   p.T = T;
-  p.start = T > 0 ? (long long)w * T / W : 0;
-  p.end = T > 0 ? (long long)(w + 1) * T / W : 0;
+  p.W = (T > 0 && T < W) ? (int)T : W;
+  p.start = (T > 0 && w < p.W) ? (long long)w * T / p.W : T;
+  p.end = (T > 0 && w < p.W) ? (long long)(w + 1) * T / p.W : T;
   p.b0 = B;
   p.P0 = T;
   if (p.start >= p.end) return p;
@@ -124,9 +127,8 @@ struct SegmentIter {
   int b;
   long long P;
 
-  __device__ SegmentIter(const WorkerPlan& plan, const int32_t* sl, int B_, int bs_, int cap_, int W_,
-                         int w_, int* st)
-      : seq_lens(sl), B(B_), bs(bs_), cap(cap_), W(W_), w(w_), status(st), p(plan), b(plan.b0), P(plan.P0) {}
+  __device__ SegmentIter(const WorkerPlan& plan, const int32_t* sl, int B_, int bs_, int cap_, int w_, int* st)
+      : seq_lens(sl), B(B_), bs(bs_), cap(cap_), W(plan.W), w(w_), status(st), p(plan), b(plan.b0), P(plan.P0) {}
 
   __device__ bool next(Segment& sg) {
     while (b < B && P < p.end) {

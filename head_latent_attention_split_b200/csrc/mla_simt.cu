@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(kThreads) simt_decode_kernel(const DecodeArgs 
   __syncthreads();
   const WorkerPlan plan = s_plan;
 
-  SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, a.W, w, a.status);
+  SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
   Segment sg;
   while (it.next(sg)) {
     const int b = sg.b;
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(32) plan_probe_kernel(const DecodeArgs a, int3
   const int w = blockIdx.x, lane = threadIdx.x;
   const int cap = a.max_blocks * a.bs;
   const WorkerPlan p = warp_plan(a.seq_lens, a.B, a.bs, cap, a.W, w, a.status);
-  SegmentIter it(p, a.seq_lens, a.B, a.bs, cap, a.W, w, a.status);
+  SegmentIter it(p, a.seq_lens, a.B, a.bs, cap, w, a.status);
   Segment sg;
   while (it.next(sg)) {
     if (sg.split == 0 && lane == 0) {

@@ -154,8 +154,8 @@ mla_status_t mla_decode_host_io(const mla_decode_params_t* params, const void* q
                                 size_t workspace_bytes, void* stream);
 
 /* Split plan on the host, for tests. Work is the flat list of cache blocks of all
- * sequences in batch order; worker w of W owns blocks [floor(w*T/W), floor((w+1)*T/W))
- * of the T blocks. Outputs (host arrays): seq_block_begin[B + 1] (prefix of blocks per
+ * sequences in batch order; with W' = min(W, T) active workers, worker w < W' owns
+ * blocks [floor(w*T/W'), floor((w+1)*T/W')) of the T blocks (at least one each). Outputs (host arrays): seq_block_begin[B + 1] (prefix of blocks per
  * sequence), seq_first_worker[B] and seq_num_splits[B] (workers that touch each
  * sequence; 0 splits for an empty sequence). W comes from mla_decode_resolve. */
 mla_status_t mla_plan_host(const mla_decode_params_t* params, const int32_t* seq_lens_host,

@@ -119,11 +119,16 @@ def test_workspace_size_formula(m):
     assert m.workspace_size(p) == al(5 * 8) + al(slots * rows * 4) + al(slots * rows * 32 * 4)
 
 
+def n_b(L, bs):
+    return (L + bs - 1) // bs
+
+
 def _plan_by_definition(lens, bs, W):
     n = [(L + bs - 1) // bs for L in lens]
     P = np.concatenate([[0], np.cumsum(n)]).astype(np.int64)
     T = int(P[-1])
-    rng = [(w * T // W, (w + 1) * T // W) for w in range(W)]
+    Wa = min(W, T) if T else W           # active workers
+    rng = [(w * T // Wa, (w + 1) * T // Wa) if w < Wa else (T, T) for w in range(W)]
     first, splits = [], []
     for b in range(len(lens)):
         touch = [w for w, (s, e) in enumerate(rng) if n[b] and s < e and s < P[b] + n[b] and e > P[b]]
@@ -132,7 +137,7 @@ def _plan_by_definition(lens, bs, W):
     return P, first, splits, rng
 
 
-@pytest.mark.parametrize("W", [1, 2, 5, 74, 300])
+@pytest.mark.parametrize("W", [1, 2, 5, 74, 300, 5000])
 def test_plan_host_matches_definition(m, W):
     rng = np.random.default_rng(W)
     lens = [int(x) for x in rng.integers(0, 3000, size=37)] + [0, 1, 64, 65, 128]
@@ -146,9 +151,13 @@ def test_plan_host_matches_definition(m, W):
     for b in range(B):
         if splits[b]:
             assert plan["first_worker"][b] == first[b]
-    # balance: worker ranges differ by at most one block
-    sizes = [e - s for s, e in ranges]
-    assert max(sizes) - min(sizes) <= 1
+    # balance: active worker ranges differ by at most one block and are never empty
+    sizes = [e - s for s, e in ranges[:min(W, int(P[-1]))]]
+    assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+    # the workers that touch a sequence are consecutive
+    for b in range(B):
+        touch = [w for w, (s, e) in enumerate(ranges) if n_b(lens[b], bs) and s < e and s < P[b] + n_b(lens[b], bs) and e > P[b]]
+        assert touch == list(range(touch[0], touch[0] + len(touch))) if touch else True
     # workspace slots w + b of all (worker, sequence) pairs are distinct and < W + B - 1
     slots = [plan["first_worker"][b] + k + b for b in range(B) if splits[b] > 1 for k in range(splits[b])]
     assert len(slots) == len(set(slots)) and (not slots or max(slots) < W + B - 1)

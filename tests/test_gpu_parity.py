@@ -157,7 +157,8 @@ def test_plan_probe_bit_exact(mla):
             exp_slot = inp["block_table"][b, tok // 64] * 64 + tok % 64
             assert np.array_equal(slot[b, :L], exp_slot)
             assert (slot[b, L:] == -1).all()
-            exp_worker = ((P[b] + tok // 64 + 1) * nw - 1) // T if L else tok
+            Wa = min(nw, T)
+            exp_worker = ((P[b] + tok // 64 + 1) * Wa - 1) // T if L else tok
             assert np.array_equal(worker[b, :L], exp_worker)
             if L:
                 assert meta[b, 0] == plan["first_worker"][b] and meta[b, 1] == plan["splits"][b]
