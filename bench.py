@@ -140,7 +140,7 @@ def cpu_oracle_rate(inp, seconds, seqs_per_step=None):
     cores = os.cpu_count() or 1
     done_bytes, elapsed, nseq = 0, 0.0, 0
     b = 0
-    while (seqs_per_step is None and elapsed < seconds and b < w.B) or (seqs_per_step and nseq < seqs_per_step):
+    while (seqs_per_step is None and elapsed < seconds and nseq < w.B) or (seqs_per_step and nseq < seqs_per_step):
         sl = slice(b, b + 1)
         t0 = time.perf_counter()
         oracle.decode(inp["q_lat"][sl], inp["q_rope"][sl], inp["kv_cache"], inp["block_table"][sl],

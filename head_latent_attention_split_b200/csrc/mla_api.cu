@@ -77,7 +77,7 @@ mla_status_t resolve(const mla_decode_params_t* p, int* kernel, int* workers) {
   const bool tc_ok = mla::tc_supported(p->kv_rank, p->rope_dim, p->block_size, p->q_dtype, p->cache_dtype,
                                        p->out_dtype, p->q_len * p->num_heads);
   int k = p->kernel;
-  if (k == MLA_KERNEL_AUTO) k = tc_ok ? MLA_KERNEL_TCGEN05 : MLA_KERNEL_SIMT;
+  if (k == MLA_KERNEL_AUTO) k = (tc_ok && mla::kTcAuto) ? MLA_KERNEL_TCGEN05 : MLA_KERNEL_SIMT;
   if (k == MLA_KERNEL_TCGEN05 && !tc_ok) return MLA_ERR_UNSUPPORTED;
   if (k == MLA_KERNEL_SIMT && !simt_ok(p)) return MLA_ERR_UNSUPPORTED;
   int W = p->num_workers;

@@ -1,9 +1,534 @@
-// Placeholder until the tcgen05 kernel lands: reports the shape as unsupported.
+// Tensor-core (tcgen05 + TMA) absorbed-MLA decode for r = 512, d_r = 64, 64-token
+// cache blocks, bf16 queries and cache.
+//
+// Design (one CTA pair = one cluster of 2 per worker and row group):
+//  * The 128 query rows of a row group (Sq * H rows of one sequence, zero-padded) are
+//    the M = 128 rows of every MMA. Their fp32 output O[128 x 512] would fill all 512
+//    TMEM columns, so the two CTAs of the pair split the latent channels: CTA j owns
+//    latent channels [256 j, 256 j + 256) and RoPE channels [32 j, 32 j + 32).
+//  * Each CTA TMA-loads only its channel slice of every 64-token cache block
+//    (4 x [64 tok][64 ch] 128B-swizzled + [64 tok][32 ch] 64B-swizzled = 36 KB per
+//    stage, 3 stages) and of the absorbed query (72 KB, once per sequence).
+//  * QK: S_j[128 x 64] = Q_j . C_j^T over the CTA's 288 channels (18 MMAs of K = 16,
+//    fp32 in TMEM). The two partial scores are exchanged through distributed shared
+//    memory (each thread ships its row, 64 floats, to the peer) and summed; both CTAs
+//    then hold the identical full score and run the identical softmax.
+//  * Online softmax in registers (thread = query row = TMEM lane), base 2, with the
+//    running maximum only moved when a tile raises it by more than 2^8, so O is
+//    rescaled rarely. P (bf16) goes to TMEM.
+//  * PV: O_j[128 x 256] += P[128 x 64] . C_j[64 x 256] with A = P from TMEM and B =
+//    the SAME shared-memory tile the QK used, read N-major (4 MMAs, N = 256).
+//  * Warp roles: warps 0-3 softmax / epilogue, warp 4 TMA producer, warp 5 TMEM
+//    allocator and single-thread MMA issuer. mbarrier pipelines between them; every
+//    wait is bounded (timeout -> MLA_ERR_TIMEOUT, clean exit).
+// The work split over workers (CTA pairs) is the flat block list plan of mla_device.cuh.
+#include <cuda.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "mla_device.cuh"
 #include "mla_tc.h"
+#include "ptx_sm100.cuh"
 
 namespace mla {
-bool tc_supported(int, int, int, int, int, int, int) { return false; }
-int tc_auto_workers(int sms, int) { return sms / 2; }
-bool tc_workers_ok(int, int) { return false; }
-cudaError_t launch_tc_decode(const DecodeArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+using namespace ptx;
+
+constexpr int kR = 512, kDR = 64, kBS = 64;
+constexpr int kRows = 128;           // query rows per row group = MMA M
+constexpr int kStages = 3;
+
+// shared memory layout, byte offsets from a 1024-aligned base
+constexpr uint32_t kQLatChunk = kRows * 128;                     // [128 rows][64 ch] bf16
+constexpr uint32_t kQRope = kRows * 64;                          // [128 rows][32 ch] bf16
+constexpr uint32_t kQBytes = 4 * kQLatChunk + kQRope;            // 73728
+constexpr uint32_t kKvLatChunk = kBS * 128;                      // [64 tok][64 ch] bf16
+constexpr uint32_t kKvRope = kBS * 64;                           // [64 tok][32 ch] bf16
+constexpr uint32_t kStageBytes = 4 * kKvLatChunk + kKvRope;      // 36864
+constexpr uint32_t kRxBytes = kRows * 64 * 4;                    // peer's partial scores
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKv = kOffQ + kQBytes;
+constexpr uint32_t kOffRx = kOffKv + kStages * kStageBytes;
+constexpr uint32_t kOffCtl = kOffRx + kRxBytes;
+constexpr uint32_t kCtlBytes = 512;
+constexpr uint32_t kSmemBytes = kOffCtl + kCtlBytes + 1024;      // + alignment slack
+
+// TMEM columns (fp32 lanes x columns; 128 lanes = 128 query rows)
+constexpr uint32_t kTmemO = 0;       // 256 columns: this CTA's output channels
+constexpr uint32_t kTmemS = 256;     // 2 x 64 columns: scores, double buffered
+constexpr uint32_t kTmemP = 384;     // 2 x 32 columns: probabilities, bf16 pairs
+constexpr uint32_t kTmemCols = 512;
+
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only if the max grows > 2^8
+
+struct Ctl {
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t q_full, q_empty;
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full[2];
+  uint64_t pv_done;
+  uint64_t rx_full;     // the peer wrote its partial scores into our rx buffer
+  uint64_t tx_ok;       // the peer consumed what we wrote into its rx buffer
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  WorkerPlan plan;
+};
+static_assert(sizeof(Ctl) <= kCtlBytes, "control block too large");
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    tc_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
+                     const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_kr,
+                     const DecodeArgs a, const int n_rg, const uint64_t timeout_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  Ctl& ctl = *reinterpret_cast<Ctl*>(smem + kOffCtl);
+  const uint32_t sQ = smem_u32(smem + kOffQ);
+  const uint32_t sKv = smem_u32(smem + kOffKv);
+  const uint32_t sRx = smem_u32(smem + kOffRx);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
+  const int cluster = (int)(blockIdx.x >> 1);
+  const int w = cluster / n_rg, rg = cluster % n_rg;
+  const int cap = a.max_blocks * a.bs;
+  volatile int* abort = &ctl.abort;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&ctl.kv_full[i]), 1);
+      mbar_init(smem_u32(&ctl.kv_empty[i]), 1);
+    }
+    mbar_init(smem_u32(&ctl.q_full), 1);
+    mbar_init(smem_u32(&ctl.q_empty), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&ctl.s_full[i]), 1);
+      mbar_init(smem_u32(&ctl.s_empty[i]), 128);
+      mbar_init(smem_u32(&ctl.p_full[i]), 128);
+    }
+    mbar_init(smem_u32(&ctl.pv_done), 1);
+    mbar_init(smem_u32(&ctl.rx_full), 128);
+    mbar_init(smem_u32(&ctl.tx_ok), 128);
+    mbar_init(smem_u32(&ctl.drain), 1);
+    ctl.abort = 0;
+    fence_mbarrier_init_cluster();
+  }
+  if (warp == kProducerWarp) {
+    const WorkerPlan p = warp_plan(a.seq_lens, a.B, a.bs, cap, a.W, w, a.status);
+    if (lane == 0) {
+      ctl.plan = p;
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_qr);
+      prefetch_tmap(&tm_kv);
+      prefetch_tmap(&tm_kr);
+    }
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(&ctl.tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  cluster_sync();          // barriers of both CTAs initialised, TMEM allocated, plan ready
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+  const WorkerPlan plan = ctl.plan;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
+      Segment sg;
+      uint32_t g = 0, seg = 0;
+      bool ok = true;
+      while (ok && it.next(sg)) {
+        ok = mbar_wait<false>(smem_u32(&ctl.q_empty), (seg & 1) ^ 1, abort, timeout_ns);
+        if (!ok) break;
+        const uint32_t qbar = smem_u32(&ctl.q_full);
+        mbar_arrive_expect_tx(qbar, kQBytes);
+        for (int c = 0; c < 4; ++c)
+          tma_load_3d(sQ + c * kQLatChunk, &tm_q, qbar, 256 * rank + 64 * c, rg * kRows, sg.b);
+        tma_load_3d(sQ + 4 * kQLatChunk, &tm_qr, qbar, 32 * rank, rg * kRows, sg.b);
+        for (int tile = sg.tile_begin; tile < sg.tile_end; ++tile, ++g) {
+          const uint32_t st = g % kStages, ph = (g / kStages) & 1;
+          ok = mbar_wait<false>(smem_u32(&ctl.kv_empty[st]), ph ^ 1, abort, timeout_ns);
+          if (!ok) break;
+          const int blk = checked_block(a.block_table, a.max_blocks, sg.b, tile, a.num_blocks, a.status);
+          const uint32_t bar = smem_u32(&ctl.kv_full[st]);
+          const uint32_t base = sKv + st * kStageBytes;
+          mbar_arrive_expect_tx(bar, kStageBytes);
+          for (int c = 0; c < 4; ++c) tma_load_3d(base + c * kKvLatChunk, &tm_kv, bar, 256 * rank + 64 * c, 0, blk);
+          tma_load_3d(base + 4 * kKvLatChunk, &tm_kr, bar, kR + 32 * rank, 0, blk);
+        }
+        ++seg;
+      }
+      // let every load already issued land before the CTA can exit
+      const uint64_t drain_ns = timeout_ns;
+      int dummy = 0;
+      for (uint32_t i = 0; i < kStages && i < g; ++i) {
+        const uint32_t gl = g - 1 - i;   // the latest load of stage gl % kStages
+        mbar_wait<false>(smem_u32(&ctl.kv_full[gl % kStages]), (gl / kStages) & 1, &dummy, drain_ns);
+      }
+      if (seg > 0) mbar_wait<false>(smem_u32(&ctl.q_full), (seg - 1) & 1, &dummy, drain_ns);
+      if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, true);
+      SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
+      Segment sg;
+      uint32_t g = 0, seg = 0;
+      bool ok = true;
+      auto issue_pv = [&](uint32_t gp, bool first) -> bool {
+        const uint32_t st = gp % kStages, pb = gp & 1;
+        if (!mbar_wait<false>(smem_u32(&ctl.p_full[pb]), (gp >> 1) & 1, abort, timeout_ns)) return false;
+        tc_fence_after();
+        const uint32_t base = sKv + st * kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          // B = C[16 tokens][256 channels], channels contiguous (N-major): 64-channel
+          // groups 8 KB apart (LBO), 8-token groups 1 KB apart (SBO)
+          const uint64_t bdesc = smem_desc(base + kk * 2048, kKvLatChunk, 1024, kSwizzle128B);
+          mma_ts(tmem + kTmemO, tmem + kTmemP + 32 * pb + 8 * kk, bdesc, idesc_pv, (first && kk == 0) ? 0u : 1u);
+        }
+        mma_commit(smem_u32(&ctl.kv_empty[st]));
+        mma_commit(smem_u32(&ctl.pv_done));
+        return true;
+      };
+      while (ok && it.next(sg)) {
+        ok = mbar_wait<false>(smem_u32(&ctl.q_full), seg & 1, abort, timeout_ns);
+        if (!ok) break;
+        tc_fence_after();
+        const int n = sg.tile_end - sg.tile_begin;
+        for (int li = 0; li < n; ++li, ++g) {
+          const uint32_t st = g % kStages, sb = g & 1;
+          ok = mbar_wait<false>(smem_u32(&ctl.kv_full[st]), (g / kStages) & 1, abort, timeout_ns) &&
+               mbar_wait<false>(smem_u32(&ctl.s_empty[sb]), ((g >> 1) & 1) ^ 1, abort, timeout_ns);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t base = sKv + st * kStageBytes;
+          const uint32_t d = tmem + kTmemS + 64 * sb;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t adesc = smem_desc(sQ + c * kQLatChunk + kk * 32, 16, 1024, kSwizzle128B);
+              const uint64_t bdesc = smem_desc(base + c * kKvLatChunk + kk * 32, 16, 1024, kSwizzle128B);
+              mma_ss(d, adesc, bdesc, idesc_qk, (c | kk) ? 1u : 0u);
+            }
+          }
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const uint64_t adesc = smem_desc(sQ + 4 * kQLatChunk + kk * 32, 16, 512, kSwizzle64B);
+            const uint64_t bdesc = smem_desc(base + 4 * kKvLatChunk + kk * 32, 16, 512, kSwizzle64B);
+            mma_ss(d, adesc, bdesc, idesc_qk, 1u);
+          }
+          mma_commit(smem_u32(&ctl.s_full[sb]));
+          if (li == n - 1) mma_commit(smem_u32(&ctl.q_empty));
+          if (li > 0) {
+            ok = issue_pv(g - 1, li == 1);
+            if (!ok) break;
+          }
+        }
+        if (!ok) break;
+        ok = issue_pv(g - 1, n == 1);
+        ++seg;
+      }
+      // every MMA issued so far completes before TMEM can be released
+      int dummy = 0;
+      mma_commit(smem_u32(&ctl.drain));
+      mbar_wait<false>(smem_u32(&ctl.drain), 0, &dummy, timeout_ns);
+      if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int row = threadIdx.x;                       // TMEM lane / query row in the group
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t rx_row = sRx + row * 256;
+    const uint32_t peer_rx_row = mapa(rx_row, peer);
+    const uint32_t peer_rx_full = mapa(smem_u32(&ctl.rx_full), peer);
+    const uint32_t peer_tx_ok = mapa(smem_u32(&ctl.tx_ok), peer);
+    const int grow = rg * kRows + row;
+    const bool valid_row = grow < a.rows;
+    const int s_idx = valid_row ? grow / a.H : 0;
+    SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
+    Segment sg;
+    uint32_t g = 0;
+    bool ok = true;
+    // waits of this role are made warp-uniform: tcgen05.ld/st below are warp-collective
+    auto wait_local = [&](uint32_t bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait<false>(bar, parity, abort, timeout_ns));
+    };
+    auto wait_peer = [&](uint32_t bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait<true>(bar, parity, abort, timeout_ns));
+    };
+    while (ok && it.next(sg)) {
+      int n_row = valid_row ? (a.causal ? sg.Lc - a.Sq + 1 + s_idx : sg.Lc) : 0;
+      if (n_row < 0) n_row = 0;
+      float m_run = -INFINITY, l_run = 0.f;
+      const int n = sg.tile_end - sg.tile_begin;
+      const int last_tile = (sg.Lc + kBS - 1) / kBS - 1;
+      for (int li = 0; li < n; ++li, ++g) {
+        const int tile = sg.tile_begin + li;
+        const uint32_t sb = g & 1;
+        ok = wait_local(smem_u32(&ctl.s_full[sb]), (g >> 1) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sv[64];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_off + kTmemS + 64 * sb + 16 * c, sv + 16 * c);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&ctl.s_empty[sb]));
+
+        // exchange partial scores with the peer CTA (rows are 256 B; 16-byte pieces are
+        // XOR-swizzled by the row to spread shared-memory banks)
+        ok = wait_peer(smem_u32(&ctl.tx_ok), (g & 1) ^ 1);
+        if (!ok) break;
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          st_cluster_v4(peer_rx_row + ((c ^ (row & 15)) << 4), __uint_as_float(sv[4 * c]),
+                        __uint_as_float(sv[4 * c + 1]), __uint_as_float(sv[4 * c + 2]),
+                        __uint_as_float(sv[4 * c + 3]));
+        mbar_arrive_remote(peer_rx_full);
+        ok = wait_peer(smem_u32(&ctl.rx_full), g & 1);
+        if (!ok) break;
+        float x[64];
+        const float4* rxp = reinterpret_cast<const float4*>(smem + kOffRx + row * 256);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float4 v = rxp[c ^ (row & 15)];
+          x[4 * c + 0] = __uint_as_float(sv[4 * c + 0]) + v.x;
+          x[4 * c + 1] = __uint_as_float(sv[4 * c + 1]) + v.y;
+          x[4 * c + 2] = __uint_as_float(sv[4 * c + 2]) + v.z;
+          x[4 * c + 3] = __uint_as_float(sv[4 * c + 3]) + v.w;
+        }
+        mbar_arrive_remote(peer_tx_ok);
+
+        // online softmax in base 2
+        const int valid = min(max(n_row - tile * kBS, 0), kBS);   // tokens of this tile the row sees
+        float mt = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+          x[k] = k < valid ? x[k] * a.scale_log2 : -INFINITY;
+          mt = fmaxf(mt, x[k]);
+        }
+        const bool grow_max = mt > m_run + kRescaleThreshold;
+        const bool rescale = grow_max && m_run != -INFINITY;
+        const float alpha = rescale ? exp2f(m_run - mt) : 1.f;
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O of this row holds earlier tiles: wait for the last PV (the one before it is
+          // known complete: it was issued before this tile's QK), scale in place
+          ok = wait_local(smem_u32(&ctl.pv_done), (g - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {
+            uint32_t v[16];
+            const uint32_t ta = tmem + lane_off + kTmemO + 16 * c;
+            tmem_ld16(ta, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+            tmem_st16(ta, v);
+          }
+          tmem_wait_st();
+        }
+        if (grow_max) {
+          l_run *= alpha;
+          m_run = mt;
+        }
+        uint32_t pk[32];
+        float psum = 0.f;
+        const bool any = m_run != -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 64; k += 2) {
+          const float p0 = any ? exp2f(x[k] - m_run) : 0.f;
+          const float p1 = any ? exp2f(x[k + 1] - m_run) : 0.f;
+          psum += p0 + p1;
+          pk[k >> 1] = pack_bf16x2(p0, p1);
+        }
+        l_run += psum;
+        const uint32_t tp = tmem + lane_off + kTmemP + 32 * sb;
+        tmem_st16(tp, pk);
+        tmem_st16(tp + 16, pk + 16);
+        tmem_wait_st();
+
+        // Slots past the sequence end in its last block may hold anything (NaN): zero
+        // those token rows of this CTA's latent slice before the PV reads them.
+        const int tail = sg.Lc % kBS;
+        if (tile == last_tile && tail != 0) {
+          const uint32_t st = g % kStages;
+          int dummy = 0;
+          mbar_wait<false>(smem_u32(&ctl.kv_full[st]), (g / kStages) & 1, &dummy, timeout_ns);
+          uint8_t* base = smem + kOffKv + st * kStageBytes;
+          const int pieces = 4 * (kBS - tail) * 8;        // 16-byte pieces
+          for (int i = row; i < pieces; i += 128) {
+            const int chunk = i / ((kBS - tail) * 8);
+            const int rem = i % ((kBS - tail) * 8);
+            const int tok = tail + rem / 8;
+            *reinterpret_cast<uint4*>(base + chunk * kKvLatChunk + tok * 128 + (rem % 8) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&ctl.p_full[sb]));
+      }
+      if (!ok) break;
+
+      // epilogue: O / l -> out (single split) or the normalised partial (several splits).
+      // Only the PV before the last tile's QK is known complete, and a parity wait only
+      // tells the last two phases apart: wait for the second-to-last PV, then the last.
+      const uint32_t gl = g - 1;
+      ok = (gl == 0 || wait_local(smem_u32(&ctl.pv_done), (gl - 1) & 1)) &&
+           wait_local(smem_u32(&ctl.pv_done), gl & 1);
+      if (!ok) break;
+      tc_fence_after();
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float lse_v = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      const size_t qrow = (size_t)sg.b * a.rows + grow;
+      const bool direct = sg.splits == 1;
+      const size_t prow = (size_t)(w + sg.b) * a.rows + grow;
+#pragma unroll 1
+      for (int c = 0; c < 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(tmem + lane_off + kTmemO + 16 * c, v);
+        tmem_wait_ld();
+        if (!valid_row) continue;
+        const int ch = 256 * (int)rank + 16 * c;
+        if (direct && a.out_dtype == kBF16) {
+          uint4 o0, o1;
+          o0.x = pack_bf16x2(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv);
+          o0.y = pack_bf16x2(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv);
+          o0.z = pack_bf16x2(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv);
+          o0.w = pack_bf16x2(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv);
+          o1.x = pack_bf16x2(__uint_as_float(v[8]) * inv, __uint_as_float(v[9]) * inv);
+          o1.y = pack_bf16x2(__uint_as_float(v[10]) * inv, __uint_as_float(v[11]) * inv);
+          o1.z = pack_bf16x2(__uint_as_float(v[12]) * inv, __uint_as_float(v[13]) * inv);
+          o1.w = pack_bf16x2(__uint_as_float(v[14]) * inv, __uint_as_float(v[15]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>((uint16_t*)a.out + qrow * kR + ch);
+          dst[0] = o0;
+          dst[1] = o1;
+        } else {
+          float* dst = direct ? (float*)a.out + qrow * kR + ch : a.o_part + prow * kR + ch;
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(dst + i) =
+                make_float4(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv,
+                            __uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
+        }
+      }
+      if (valid_row && rank == 0) {
+        if (direct)
+          a.lse[qrow] = lse_v;
+        else
+          a.lse_part[prow] = lse_v;
+      }
+      if (sg.split == 0 && rg == 0 && rank == 0 && row == 0) {
+        a.meta[2 * sg.b] = sg.first_worker;
+        a.meta[2 * sg.b + 1] = sg.splits;
+      }
+      tc_fence_before();
+    }
+    if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
+  }
+
+  // ------------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  cluster_sync();   // no CTA leaves while its peer may still touch its shared memory
+}
+
+// ---------------------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map: dims (inner -> outer), byte strides of dims 1 and 2, box.
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                 uint64_t s2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1, s2};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int row_groups(int rows) { return (rows + kRows - 1) / kRows; }
+
+}  // namespace
+
+bool tc_supported(int r, int d_r, int block_size, int q_dtype, int cache_dtype, int out_dtype, int rows) {
+  return r == kR && d_r == kDR && block_size == kBS && q_dtype == kBF16 && cache_dtype == kBF16 &&
+         (out_dtype == kBF16 || out_dtype == kF32) && rows >= 1 && row_groups(rows) <= 1024;
+}
+
+int tc_auto_workers(int sms, int rows) {
+  const int w = sms / (2 * row_groups(rows));
+  return w > 0 ? w : 1;
+}
+
+bool tc_workers_ok(int W, int rows) { return W >= 1 && (long long)W * row_groups(rows) * 2 <= 65535; }
+
+cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
+  const int n_rg = row_groups(a.rows);
+  CUtensorMap tq, tqr, tkv, tkr;
+  const uint64_t rows = (uint64_t)a.rows;
+  if (!make_map_3d(&tq, a.q_lat, kR, rows, a.B, kR * 2, rows * kR * 2, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_3d(&tqr, a.q_rope, kDR, rows, a.B, kDR * 2, rows * kDR * 2, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_3d(&tkv, a.cache, kR + kDR, kBS, a.num_blocks, (kR + kDR) * 2, (uint64_t)kBS * (kR + kDR) * 2, 64,
+                   kBS, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_3d(&tkr, a.cache, kR + kDR, kBS, a.num_blocks, (kR + kDR) * 2, (uint64_t)kBS * (kR + kDR) * 2, 32,
+                   kBS, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  static std::once_flag attr_once[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once[dev & 63], [&] {
+    attr_err = cudaFuncSetAttribute(tc_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  const uint64_t timeout_ns = 2000000000ull;
+  const dim3 grid(2 * a.W * n_rg);
+  tc_decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tqr, tkv, tkr, a, n_rg, timeout_ns);
+  return cudaGetLastError();
+}
+
 }  // namespace mla

@@ -5,6 +5,9 @@
 
 namespace mla {
 
+// Whether MLA_KERNEL_AUTO picks the tensor-core kernel for the shapes it supports.
+constexpr bool kTcAuto = false;
+
 // True when the tensor-core kernel handles this problem (rows = Sq * H).
 bool tc_supported(int r, int d_r, int block_size, int q_dtype, int cache_dtype, int out_dtype, int rows);
 // Default worker count for `sms` SMs.
