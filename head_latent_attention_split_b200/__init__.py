@@ -8,5 +8,6 @@ this package is a thin binding over it.
 """
 from .binding import (BF16, E4M3, F32, KERNELS, MlaError, Params, abi_version, device_status,  # noqa: F401
                       host_io_workspace_size, make_params, mla_decode, mla_decode_host_io, mla_decode_timed, plan_host,
+                      mla_decode_noalloc, noalloc_max_workspace,
                       plan_probe, resolve, status_string, workspace_size)
 from .api import decode, decode_host_io, params_for  # noqa: F401

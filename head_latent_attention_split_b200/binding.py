@@ -25,7 +25,8 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "M
 
 EXPORTED = ("mla_decode_workspace_size", "mla_decode_resolve", "mla_decode", "mla_decode_timed",
             "mla_decode_host_io_workspace_size", "mla_decode_host_io", "mla_plan_host", "mla_plan_probe",
-            "mla_get_device_status", "mla_status_string", "mla_abi_version")
+            "mla_get_device_status", "mla_status_string", "mla_abi_version", "mla_decode_noalloc",
+            "mla_decode_noalloc_max_workspace")
 
 
 class MlaError(RuntimeError):
@@ -56,6 +57,9 @@ def _load():
     L.mla_decode_timed.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.POINTER(vp)]
     L.mla_decode_host_io_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
     L.mla_decode_host_io.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.mla_decode_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.mla_decode_noalloc_max_workspace.argtypes = []
+    L.mla_decode_noalloc_max_workspace.restype = ctypes.c_size_t
     L.mla_plan_host.argtypes = [P, vp, vp, vp, vp]
     L.mla_plan_probe.argtypes = [P, vp, vp, vp, vp, vp, vp]
     L.mla_get_device_status.argtypes = [vp, i32p]
@@ -66,7 +70,7 @@ def _load():
         if not hasattr(L, name):
             raise ImportError(f"{LIB_PATH} lacks {name}: rebuild it")
         f = getattr(L, name)
-        if f.restype is ctypes.c_int:   # default
+        if f.restype is ctypes.c_int and name != "mla_decode_noalloc_max_workspace":   # default
             f.restype = ctypes.c_int32
     L.mla_status_string.restype = ctypes.c_char_p
     return L
@@ -176,6 +180,21 @@ def mla_decode_host_io(p: Params, q_lat_host, q_rope_host, kv_cache, k_rope_cach
     if check:
         _check(st, "mla_decode_host_io")
     return st
+
+
+def mla_decode_noalloc(p: Params, q_lat, q_rope, kv_cache, k_rope_cache, kv_scale, block_table, seq_lens, out,
+                       lse, stream=None, check=True) -> int:
+    """C-ABI call that takes no workspace: the library's own device scratch array is used."""
+    st = lib.mla_decode_noalloc(ctypes.byref(p), _addr(q_lat), _addr(q_rope), _addr(kv_cache), _addr(k_rope_cache),
+                                _addr(kv_scale), _addr(block_table), _addr(seq_lens), _addr(out), _addr(lse),
+                                _stream(stream))
+    if check:
+        _check(st, "mla_decode_noalloc")
+    return st
+
+
+def noalloc_max_workspace() -> int:
+    return lib.mla_decode_noalloc_max_workspace()
 
 
 def device_status(stream=None) -> int:

@@ -153,6 +153,28 @@ mla_status_t mla_decode_host_io(const mla_decode_params_t* params, const void* q
                                 void* out_host, float* lse_host, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* Largest workspace, in bytes, that mla_decode_noalloc can serve (64 MiB). */
+#define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* mla_decode for callers that cannot allocate device memory on the decode path (a
+ * serving engine that has reserved the GPU's memory for its cache, a plugin running in
+ * a memory pool it does not own). The paper has no counterpart to this entry point: it
+ * is a convenience of the library, not a step of the method. The split workspace is a file-scope device array of
+ * MLA_NOALLOC_SCRATCH_BYTES that every GPU loading the library keeps until exit.
+ * Arguments are those of mla_decode without the workspace. The first call on each
+ * device looks up that device's array address (make it before any stream capture).
+ * Returns MLA_ERR_WORKSPACE_TOO_SMALL, with nothing launched, when
+ * mla_decode_workspace_size() exceeds MLA_NOALLOC_SCRATCH_BYTES. Allocates nothing.
+ * All calls on a device share the array: calls whose GPU work overlaps race, so
+ * serialise them (one stream, or external ordering). */
+mla_status_t mla_decode_noalloc(const mla_decode_params_t* params, const void* q_lat, const void* q_rope,
+                                const void* kv_cache, const void* k_rope_cache, const float* kv_scale,
+                                const int32_t* block_table, const int32_t* seq_lens, void* out, float* lse,
+                                void* stream);
+
+/* MLA_NOALLOC_SCRATCH_BYTES as compiled into the loaded library. */
+size_t mla_decode_noalloc_max_workspace(void);
+
 /* Split plan on the host, for tests. Work is the flat list of cache blocks of all
  * sequences in batch order; with W' = min(W, T) active workers, worker w < W' owns
  * blocks [floor(w*T/W'), floor((w+1)*T/W')) of the T blocks (at least one each). Outputs (host arrays): seq_block_begin[B + 1] (prefix of blocks per
