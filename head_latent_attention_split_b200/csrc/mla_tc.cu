@@ -74,7 +74,7 @@ struct Ctl {
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2];
   uint64_t pv_done;
-  uint64_t rx_full;     // the peer wrote its partial scores into our rx buffer
+  uint64_t rx_full;     // the peer's partial scores (32 KB of st.async) landed in our rx buffer
   uint64_t tx_ok;       // the peer consumed what we wrote into its rx buffer
   uint64_t drain;
   uint32_t tmem_base;
@@ -120,8 +120,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&ctl.p_full[i]), 128);
     }
     mbar_init(smem_u32(&ctl.pv_done), 1);
-    mbar_init(smem_u32(&ctl.rx_full), 128);
-    mbar_init(smem_u32(&ctl.tx_ok), 128);
+    mbar_init(smem_u32(&ctl.rx_full), 1);    // armed locally, completed by the peer's st.async bytes
+    mbar_init(smem_u32(&ctl.tx_ok), 4);      // one arrival per softmax warp of the peer
     mbar_init(smem_u32(&ctl.drain), 1);
     ctl.abort = 0;
     fence_mbarrier_init_cluster();
@@ -297,14 +297,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
         // exchange partial scores with the peer CTA (rows are 256 B; 16-byte pieces are
         // XOR-swizzled by the row to spread shared-memory banks)
+        if (row == 0) mbar_arrive_expect_tx(smem_u32(&ctl.rx_full), kRxBytes);   // arm this tile's phase
         ok = wait_peer(smem_u32(&ctl.tx_ok), (g & 1) ^ 1);
         if (!ok) break;
 #pragma unroll
         for (int c = 0; c < 16; ++c)
-          st_cluster_v4(peer_rx_row + ((c ^ (row & 15)) << 4), __uint_as_float(sv[4 * c]),
-                        __uint_as_float(sv[4 * c + 1]), __uint_as_float(sv[4 * c + 2]),
-                        __uint_as_float(sv[4 * c + 3]));
-        mbar_arrive_remote(peer_rx_full);
+          st_async_v4(peer_rx_row + ((c ^ (row & 15)) << 4), sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3],
+                      peer_rx_full);
         ok = wait_peer(smem_u32(&ctl.rx_full), g & 1);
         if (!ok) break;
         float x[64];
@@ -317,7 +316,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           x[4 * c + 2] = __uint_as_float(sv[4 * c + 2]) + v.z;
           x[4 * c + 3] = __uint_as_float(sv[4 * c + 3]) + v.w;
         }
-        mbar_arrive_remote(peer_tx_ok);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(peer_tx_ok);     // this warp's rows of our rx are consumed
 
         // online softmax in base 2
         const int valid = min(max(n_row - tile * kBS, 0), kBS);   // tokens of this tile the row sees
@@ -329,7 +329,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         const bool grow_max = mt > m_run + kRescaleThreshold;
         const bool rescale = grow_max && m_run != -INFINITY;
-        const float alpha = rescale ? exp2f(m_run - mt) : 1.f;
+        const float alpha = rescale ? ex2_approx(m_run - mt) : 1.f;
         if (__any_sync(0xffffffffu, rescale)) {
           // O of this row holds earlier tiles: wait for the last PV (the one before it is
           // known complete: it was issued before this tile's QK), scale in place
@@ -357,8 +357,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const bool any = m_run != -INFINITY;
 #pragma unroll
         for (int k = 0; k < 64; k += 2) {
-          const float p0 = any ? exp2f(x[k] - m_run) : 0.f;
-          const float p1 = any ? exp2f(x[k + 1] - m_run) : 0.f;
+          const float p0 = any ? ex2_approx(x[k] - m_run) : 0.f;
+          const float p1 = any ? ex2_approx(x[k + 1] - m_run) : 0.f;
           psum += p0 + p1;
           pk[k >> 1] = pack_bf16x2(p0, p1);
         }

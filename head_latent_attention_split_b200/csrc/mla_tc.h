@@ -6,7 +6,7 @@
 namespace mla {
 
 // Whether MLA_KERNEL_AUTO picks the tensor-core kernel for the shapes it supports.
-constexpr bool kTcAuto = false;
+constexpr bool kTcAuto = true;
 
 // True when the tensor-core kernel handles this problem (rows = Sq * H).
 bool tc_supported(int r, int d_r, int block_size, int q_dtype, int cache_dtype, int out_dtype, int rows);
