@@ -1,25 +1,38 @@
 // Tensor-core (tcgen05 + TMA) absorbed-MLA decode for r = 512, d_r = 64, 64-token
-// cache blocks, bf16 queries and cache.
+// cache blocks, bf16 queries, bf16 cache.
 //
 // Design (one CTA pair = one cluster of 2 per worker and row group):
 //  * The 128 query rows of a row group (Sq * H rows of one sequence, zero-padded) are
 //    the M = 128 rows of every MMA. Their fp32 output O[128 x 512] would fill all 512
 //    TMEM columns, so the two CTAs of the pair split the latent channels: CTA j owns
 //    latent channels [256 j, 256 j + 256) and RoPE channels [32 j, 32 j + 32).
+//  * TMEM per CTA (128 lanes = query rows): O [0, 256), scores S [256, 320),
+//    probabilities P (bf16 pairs, double buffered) [320, 384), and the CTA's half of
+//    the absorbed query, latent part, as a TMEM A operand [384, 512).
 //  * Each CTA TMA-loads only its channel slice of every 64-token cache block
 //    (4 x [64 tok][64 ch] 128B-swizzled + [64 tok][32 ch] 64B-swizzled = 36 KB per
-//    stage, 3 stages) and of the absorbed query (72 KB, once per sequence).
-//  * QK: S_j[128 x 64] = Q_j . C_j^T over the CTA's 288 channels (18 MMAs of K = 16,
-//    fp32 in TMEM). The two partial scores are exchanged through distributed shared
-//    memory (each thread ships its row, 64 floats, to the peer) and summed; both CTAs
-//    then hold the identical full score and run the identical softmax.
-//  * Online softmax in registers (thread = query row = TMEM lane), base 2, with the
-//    running maximum only moved when a tile raises it by more than 2^8, so O is
-//    rescaled rarely. P (bf16) goes to TMEM.
+//    stage, 4 stages). The query's RoPE part stays in shared memory (8 KB).
+//  * QK: S_j[128 x 64] = Q_j . C_j^T over the CTA's 288 channels (16 MMAs with A in
+//    TMEM + 2 with A in shared memory, K = 16 each).
+//  * Score exchange: the 8 softmax warps each own 32 rows x 32 columns of S. A warp
+//    stages its fp32 partial scores (4 KB) in shared memory and ships them with one
+//    bulk copy into the peer CTA, completing bytes on the peer's mbarrier; the peer's
+//    matching warp adds the two partials in the same order, so both CTAs hold the same
+//    full score. Two 32 KB buffers alternate roles: the one that received tile t - 1
+//    stages the outgoing partials of tile t + 1... precisely, buffer t & 1 receives
+//    tile t and buffer (t + 1) & 1 stages tile t; per-warp mbarriers tell the sender
+//    when the peer's buffer is free again.
+//  * Software pipeline of the softmax warps, iteration g: load S(g) and ship it;
+//    finish tile g - 1 (exponentials, P into TMEM); then combine tile g's partials and
+//    take its row maximum. The exchange of tile g overlaps the exponentials of g - 1.
+//    Two threads per query row (32 columns each) exchange their maxima through shared
+//    memory; the running maximum only moves when a tile raises it by more than 2^8,
+//    so O is rescaled rarely.
 //  * PV: O_j[128 x 256] += P[128 x 64] . C_j[64 x 256] with A = P from TMEM and B =
-//    the SAME shared-memory tile the QK used, read N-major (4 MMAs, N = 256).
-//  * Warp roles: warps 0-3 softmax / epilogue, warp 4 TMA producer, warp 5 TMEM
-//    allocator and single-thread MMA issuer. mbarrier pipelines between them; every
+//    the SAME shared-memory tile the QK used, read N-major (4 MMAs, N = 256). The MMA
+//    issuer runs QK(k) then PV(k - 2).
+//  * Warp roles: warps 0-7 softmax / epilogue, warp 8 TMA producer, warp 9 TMEM
+//    allocator and single-thread MMA issuer; mbarrier pipelines between them. Every
 //    wait is bounded (timeout -> MLA_ERR_TIMEOUT, clean exit).
 // The work split over workers (CTA pairs) is the flat block list plan of mla_device.cuh.
 #include <cuda.h>
@@ -38,32 +51,35 @@ using namespace ptx;
 
 constexpr int kR = 512, kDR = 64, kBS = 64;
 constexpr int kRows = 128;           // query rows per row group = MMA M
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 
 // shared memory layout, byte offsets from a 1024-aligned base
-constexpr uint32_t kQLatChunk = kRows * 128;                     // [128 rows][64 ch] bf16
-constexpr uint32_t kQRope = kRows * 64;                          // [128 rows][32 ch] bf16
-constexpr uint32_t kQBytes = 4 * kQLatChunk + kQRope;            // 73728
-constexpr uint32_t kKvLatChunk = kBS * 128;                      // [64 tok][64 ch] bf16
-constexpr uint32_t kKvRope = kBS * 64;                           // [64 tok][32 ch] bf16
+constexpr uint32_t kKvLatChunk = kBS * 128;                      // [64 tok][64 ch] bf16, 128B swizzle
+constexpr uint32_t kKvRope = kBS * 64;                           // [64 tok][32 ch] bf16, 64B swizzle
 constexpr uint32_t kStageBytes = 4 * kKvLatChunk + kKvRope;      // 36864
-constexpr uint32_t kRxBytes = kRows * 64 * 4;                    // peer's partial scores
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKv = kOffQ + kQBytes;
-constexpr uint32_t kOffRx = kOffKv + kStages * kStageBytes;
-constexpr uint32_t kOffCtl = kOffRx + kRxBytes;
-constexpr uint32_t kCtlBytes = 512;
+constexpr uint32_t kQRope = kRows * 64;                          // [128 rows][32 ch] bf16, 64B swizzle
+constexpr uint32_t kXBytes = kRows * 64 * 4;                     // partial scores [128 rows][64] fp32
+constexpr uint32_t kXChunk = kXBytes / 8;                        // one softmax warp's 32 rows x 32 cols
+constexpr uint32_t kOffKv = 0;
+constexpr uint32_t kOffQr = kOffKv + kStages * kStageBytes;
+constexpr uint32_t kOffX = kOffQr + kQRope;                      // two exchange buffers
+constexpr uint32_t kOffCtl = kOffX + 2 * kXBytes;
+constexpr uint32_t kCtlBytes = 4096;
 constexpr uint32_t kSmemBytes = kOffCtl + kCtlBytes + 1024;      // + alignment slack
+static_assert(kOffQr % 1024 == 0 && kOffX % 1024 == 0, "buffers need 1024-byte alignment");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// TMEM columns (fp32 lanes x columns; 128 lanes = 128 query rows)
-constexpr uint32_t kTmemO = 0;       // 256 columns: this CTA's output channels
-constexpr uint32_t kTmemS = 256;     // 2 x 64 columns: scores, double buffered
-constexpr uint32_t kTmemP = 384;     // 2 x 32 columns: probabilities, bf16 pairs
+// TMEM columns (32-bit lanes x columns; lane = query row)
+constexpr uint32_t kTmemO = 0;       // 256: this CTA's output channels
+constexpr uint32_t kTmemS = 256;     // 64: scores of the current tile
+constexpr uint32_t kTmemP = 320;     // 2 x 32: probabilities, bf16 pairs
+constexpr uint32_t kTmemQ = 384;     // 128: absorbed query, this CTA's 256 latent channels
 constexpr uint32_t kTmemCols = 512;
 
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kSoftmaxThreads = 256;  // warps 0-7
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only if the max grows > 2^8
 
@@ -71,15 +87,19 @@ struct Ctl {
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
   uint64_t q_full, q_empty;
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full, s_empty;
   uint64_t p_full[2];
-  uint64_t pv_done;
-  uint64_t rx_full;     // the peer's partial scores (32 KB of st.async) landed in our rx buffer
-  uint64_t tx_ok;       // the peer consumed what we wrote into its rx buffer
+  uint64_t pv_done[2];      // PV of tile t completes a phase of pv_done[t & 1]
+  uint64_t rx_full[2];      // exchange buffer b holds the peer's partials of the next tile t, t & 1 == b
+  uint64_t tx_ok[8][2];     // per warp: the peer's buffer b may take our next partials
+  uint64_t mx[4];           // the two warps sharing 32 rows published their tile maxima
+  uint64_t lx[4];           // ... their row sums
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
   WorkerPlan plan;
+  float mbuf[2][2][kRows];  // [tile parity][half][row]
+  float lbuf[2][kRows];     // [half][row]
 };
 static_assert(sizeof(Ctl) <= kCtlBytes, "control block too large");
 
@@ -90,15 +110,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    tc_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qr,
-                     const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_kr,
-                     const DecodeArgs a, const int n_rg, const uint64_t timeout_ns) {
+    tc_decode_kernel(const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_kv,
+                     const __grid_constant__ CUtensorMap tm_kr, const DecodeArgs a, const int n_rg,
+                     const uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   Ctl& ctl = *reinterpret_cast<Ctl*>(smem + kOffCtl);
-  const uint32_t sQ = smem_u32(smem + kOffQ);
   const uint32_t sKv = smem_u32(smem + kOffKv);
-  const uint32_t sRx = smem_u32(smem + kOffRx);
+  const uint32_t sQr = smem_u32(smem + kOffQr);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
@@ -112,16 +131,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&ctl.kv_full[i]), 1);
       mbar_init(smem_u32(&ctl.kv_empty[i]), 1);
     }
-    mbar_init(smem_u32(&ctl.q_full), 1);
+    mbar_init(smem_u32(&ctl.q_full), 1 + kSoftmaxThreads);   // RoPE part by TMA + latent part into TMEM
     mbar_init(smem_u32(&ctl.q_empty), 1);
+    mbar_init(smem_u32(&ctl.s_full), 1);
+    mbar_init(smem_u32(&ctl.s_empty), kSoftmaxThreads);
+    for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&ctl.p_full[i]), kSoftmaxThreads);
+    for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&ctl.pv_done[i]), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&ctl.s_full[i]), 1);
-      mbar_init(smem_u32(&ctl.s_empty[i]), 128);
-      mbar_init(smem_u32(&ctl.p_full[i]), 128);
+      mbar_init(smem_u32(&ctl.rx_full[i]), 1);
+      mbar_arrive_expect_tx(smem_u32(&ctl.rx_full[i]), kXBytes);   // armed for tiles 0 and 1
     }
-    mbar_init(smem_u32(&ctl.pv_done), 1);
-    mbar_init(smem_u32(&ctl.rx_full), 1);    // armed locally, completed by the peer's st.async bytes
-    mbar_init(smem_u32(&ctl.tx_ok), 4);      // one arrival per softmax warp of the peer
+    for (int i = 0; i < 8; ++i)
+      for (int j = 0; j < 2; ++j) mbar_init(smem_u32(&ctl.tx_ok[i][j]), 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(smem_u32(&ctl.mx[i]), 64);
+      mbar_init(smem_u32(&ctl.lx[i]), 64);
+    }
     mbar_init(smem_u32(&ctl.drain), 1);
     ctl.abort = 0;
     fence_mbarrier_init_cluster();
@@ -130,7 +155,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const WorkerPlan p = warp_plan(a.seq_lens, a.B, a.bs, cap, a.W, w, a.status);
     if (lane == 0) {
       ctl.plan = p;
-      prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_qr);
       prefetch_tmap(&tm_kv);
       prefetch_tmap(&tm_kr);
@@ -157,10 +181,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ok = mbar_wait<false>(smem_u32(&ctl.q_empty), (seg & 1) ^ 1, abort, timeout_ns);
         if (!ok) break;
         const uint32_t qbar = smem_u32(&ctl.q_full);
-        mbar_arrive_expect_tx(qbar, kQBytes);
-        for (int c = 0; c < 4; ++c)
-          tma_load_3d(sQ + c * kQLatChunk, &tm_q, qbar, 256 * rank + 64 * c, rg * kRows, sg.b);
-        tma_load_3d(sQ + 4 * kQLatChunk, &tm_qr, qbar, 32 * rank, rg * kRows, sg.b);
+        mbar_arrive_expect_tx(qbar, kQRope);
+        tma_load_3d(sQr, &tm_qr, qbar, 32 * rank, rg * kRows, sg.b);
         for (int tile = sg.tile_begin; tile < sg.tile_end; ++tile, ++g) {
           const uint32_t st = g % kStages, ph = (g / kStages) & 1;
           ok = mbar_wait<false>(smem_u32(&ctl.kv_empty[st]), ph ^ 1, abort, timeout_ns);
@@ -175,13 +197,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ++seg;
       }
       // let every load already issued land before the CTA can exit
-      const uint64_t drain_ns = timeout_ns;
       int dummy = 0;
       for (uint32_t i = 0; i < kStages && i < g; ++i) {
         const uint32_t gl = g - 1 - i;   // the latest load of stage gl % kStages
-        mbar_wait<false>(smem_u32(&ctl.kv_full[gl % kStages]), (gl / kStages) & 1, &dummy, drain_ns);
+        mbar_wait<false>(smem_u32(&ctl.kv_full[gl % kStages]), (gl / kStages) & 1, &dummy, timeout_ns);
       }
-      if (seg > 0) mbar_wait<false>(smem_u32(&ctl.q_full), (seg - 1) & 1, &dummy, drain_ns);
       if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
     }
   } else if (warp == kMmaWarp) {
@@ -206,46 +226,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           mma_ts(tmem + kTmemO, tmem + kTmemP + 32 * pb + 8 * kk, bdesc, idesc_pv, (first && kk == 0) ? 0u : 1u);
         }
         mma_commit(smem_u32(&ctl.kv_empty[st]));
-        mma_commit(smem_u32(&ctl.pv_done));
+        mma_commit(smem_u32(&ctl.pv_done[pb]));
         return true;
       };
       while (ok && it.next(sg)) {
         ok = mbar_wait<false>(smem_u32(&ctl.q_full), seg & 1, abort, timeout_ns);
         if (!ok) break;
         tc_fence_after();
+        const uint32_t g0 = g;
         const int n = sg.tile_end - sg.tile_begin;
         for (int li = 0; li < n; ++li, ++g) {
-          const uint32_t st = g % kStages, sb = g & 1;
+          const uint32_t st = g % kStages;
           ok = mbar_wait<false>(smem_u32(&ctl.kv_full[st]), (g / kStages) & 1, abort, timeout_ns) &&
-               mbar_wait<false>(smem_u32(&ctl.s_empty[sb]), ((g >> 1) & 1) ^ 1, abort, timeout_ns);
+               mbar_wait<false>(smem_u32(&ctl.s_empty), (g & 1) ^ 1, abort, timeout_ns);
           if (!ok) break;
           tc_fence_after();
           const uint32_t base = sKv + st * kStageBytes;
-          const uint32_t d = tmem + kTmemS + 64 * sb;
+          const uint32_t d = tmem + kTmemS;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t adesc = smem_desc(sQ + c * kQLatChunk + kk * 32, 16, 1024, kSwizzle128B);
-              const uint64_t bdesc = smem_desc(base + c * kKvLatChunk + kk * 32, 16, 1024, kSwizzle128B);
-              mma_ss(d, adesc, bdesc, idesc_qk, (c | kk) ? 1u : 0u);
-            }
+          for (int kk = 0; kk < 16; ++kk) {
+            // latent channels [16 kk, 16 kk + 16): A = Q from TMEM, B = the cache chunk
+            const uint64_t bdesc = smem_desc(base + (kk >> 2) * kKvLatChunk + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+            mma_ts(d, tmem + kTmemQ + 8 * kk, bdesc, idesc_qk, kk ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
-            const uint64_t adesc = smem_desc(sQ + 4 * kQLatChunk + kk * 32, 16, 512, kSwizzle64B);
+            const uint64_t adesc = smem_desc(sQr + kk * 32, 16, 512, kSwizzle64B);
             const uint64_t bdesc = smem_desc(base + 4 * kKvLatChunk + kk * 32, 16, 512, kSwizzle64B);
             mma_ss(d, adesc, bdesc, idesc_qk, 1u);
           }
-          mma_commit(smem_u32(&ctl.s_full[sb]));
+          mma_commit(smem_u32(&ctl.s_full));
           if (li == n - 1) mma_commit(smem_u32(&ctl.q_empty));
-          if (li > 0) {
-            ok = issue_pv(g - 1, li == 1);
+          if (li >= 2) {
+            ok = issue_pv(g - 2, li == 2);
             if (!ok) break;
           }
         }
         if (!ok) break;
-        ok = issue_pv(g - 1, n == 1);
+        for (int li = n >= 2 ? n - 2 : 0; ok && li < n; ++li) ok = issue_pv(g0 + li, li == 0);
         ++seg;
       }
       // every MMA issued so far completes before TMEM can be released
@@ -256,18 +274,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    const int row = threadIdx.x;                       // TMEM lane / query row in the group
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint32_t rx_row = sRx + row * 256;
-    const uint32_t peer_rx_row = mapa(rx_row, peer);
-    const uint32_t peer_rx_full = mapa(smem_u32(&ctl.rx_full), peer);
-    const uint32_t peer_tx_ok = mapa(smem_u32(&ctl.tx_ok), peer);
+    const int st_idx = threadIdx.x;                    // 0..255
+    const int row = st_idx & (kRows - 1);              // TMEM lane / query row in the group
+    const int half = st_idx >> 7;                      // columns [32 half, 32 half + 32)
+    const int quad = warp & 3;                         // the TMEM lane quarter of this warp
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    // exchange: this warp's 4 KB chunk of an exchange buffer; 16-byte pieces of a lane's
+    // 128-byte row XOR-swizzled by the lane to spread shared-memory banks
+    const uint32_t chunk_off = kOffX + warp * kXChunk + lane * 128;
+    const uint32_t peer_x0 = mapa(smem_u32(smem + kOffX + warp * kXChunk), peer);
+    const uint32_t peer_rx_full0 = mapa(smem_u32(&ctl.rx_full[0]), peer);
+    const uint32_t peer_rx_full1 = mapa(smem_u32(&ctl.rx_full[1]), peer);
+    const uint32_t peer_tx_ok0 = mapa(smem_u32(&ctl.tx_ok[warp][0]), peer);
+    const uint32_t peer_tx_ok1 = mapa(smem_u32(&ctl.tx_ok[warp][1]), peer);
     const int grow = rg * kRows + row;
     const bool valid_row = grow < a.rows;
     const int s_idx = valid_row ? grow / a.H : 0;
+    const float scale_log2 = a.scale_log2;
     SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
     Segment sg;
-    uint32_t g = 0;
+    uint32_t g = 0, seg = 0;
     bool ok = true;
     // waits of this role are made warp-uniform: tcgen05.ld/st below are warp-collective
     auto wait_local = [&](uint32_t bar, uint32_t parity) {
@@ -276,141 +302,194 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto wait_peer = [&](uint32_t bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait<true>(bar, parity, abort, timeout_ns));
     };
+    // PV(j) done. Valid while PV(j - 2) is complete and PV(j + 2) cannot be (its P is
+    // not written yet): callers only wait for PVs of the current segment.
+    auto wait_pv = [&](uint32_t j) { return wait_local(smem_u32(&ctl.pv_done[j & 1]), (j >> 1) & 1); };
     while (ok && it.next(sg)) {
+      // this segment's absorbed query, latent half of this CTA, into TMEM
+      ok = wait_local(smem_u32(&ctl.q_empty), (seg & 1) ^ 1);
+      if (!ok) break;
+      {
+        uint32_t qv[64];
+        const uint4* src = reinterpret_cast<const uint4*>((const uint16_t*)a.q_lat +
+                                                         ((size_t)sg.b * a.rows + (valid_row ? grow : 0)) * kR +
+                                                         256 * rank + 128 * half);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint4 v = valid_row ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+          qv[4 * i] = v.x;
+          qv[4 * i + 1] = v.y;
+          qv[4 * i + 2] = v.z;
+          qv[4 * i + 3] = v.w;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_st16(tmem + lane_off + kTmemQ + 64 * half + 16 * c, qv + 16 * c);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&ctl.q_full));
+      }
       int n_row = valid_row ? (a.causal ? sg.Lc - a.Sq + 1 + s_idx : sg.Lc) : 0;
       if (n_row < 0) n_row = 0;
       float m_run = -INFINITY, l_run = 0.f;
       const int n = sg.tile_end - sg.tile_begin;
       const int last_tile = (sg.Lc + kBS - 1) / kBS - 1;
-      for (int li = 0; li < n; ++li, ++g) {
-        const int tile = sg.tile_begin + li;
-        const uint32_t sb = g & 1;
-        ok = wait_local(smem_u32(&ctl.s_full[sb]), (g >> 1) & 1);
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t sv[64];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld16(tmem + lane_off + kTmemS + 64 * sb + 16 * c, sv + 16 * c);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(smem_u32(&ctl.s_empty[sb]));
-
-        // exchange partial scores with the peer CTA (rows are 256 B; 16-byte pieces are
-        // XOR-swizzled by the row to spread shared-memory banks)
-        if (row == 0) mbar_arrive_expect_tx(smem_u32(&ctl.rx_full), kRxBytes);   // arm this tile's phase
-        ok = wait_peer(smem_u32(&ctl.tx_ok), (g & 1) ^ 1);
-        if (!ok) break;
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          st_async_v4(peer_rx_row + ((c ^ (row & 15)) << 4), sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3],
-                      peer_rx_full);
-        ok = wait_peer(smem_u32(&ctl.rx_full), g & 1);
-        if (!ok) break;
-        float x[64];
-        const float4* rxp = reinterpret_cast<const float4*>(smem + kOffRx + row * 256);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float4 v = rxp[c ^ (row & 15)];
-          x[4 * c + 0] = __uint_as_float(sv[4 * c + 0]) + v.x;
-          x[4 * c + 1] = __uint_as_float(sv[4 * c + 1]) + v.y;
-          x[4 * c + 2] = __uint_as_float(sv[4 * c + 2]) + v.z;
-          x[4 * c + 3] = __uint_as_float(sv[4 * c + 3]) + v.w;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(peer_tx_ok);     // this warp's rows of our rx are consumed
-
-        // online softmax in base 2
-        const int valid = min(max(n_row - tile * kBS, 0), kBS);   // tokens of this tile the row sees
-        float mt = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          x[k] = k < valid ? x[k] * a.scale_log2 : -INFINITY;
-          mt = fmaxf(mt, x[k]);
-        }
-        const bool grow_max = mt > m_run + kRescaleThreshold;
-        const bool rescale = grow_max && m_run != -INFINITY;
-        const float alpha = rescale ? ex2_approx(m_run - mt) : 1.f;
-        if (__any_sync(0xffffffffu, rescale)) {
-          // O of this row holds earlier tiles: wait for the last PV (the one before it is
-          // known complete: it was issued before this tile's QK), scale in place
-          ok = wait_local(smem_u32(&ctl.pv_done), (g - 1) & 1);
+      float x[32];          // scaled scores (log2 units) of the tile awaiting its exponentials
+      float mt = -INFINITY; // that tile's row maximum
+      for (int li = 0; li <= n; ++li) {
+        const uint32_t gt = g + li;   // tile of stage A / B1 (g + li), B2 handles gt - 1
+        uint32_t sv[32];
+        if (li < n) {
+          // ---- A: scores of tile gt out of TMEM, staged and shipped to the peer
+          ok = wait_local(smem_u32(&ctl.s_full), gt & 1);
           if (!ok) break;
           tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < 16; ++c) {
-            uint32_t v[16];
-            const uint32_t ta = tmem + lane_off + kTmemO + 16 * c;
-            tmem_ld16(ta, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-            tmem_st16(ta, v);
+          tmem_ld16(tmem + lane_off + kTmemS + 32 * half, sv);
+          tmem_ld16(tmem + lane_off + kTmemS + 32 * half + 16, sv + 16);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(smem_u32(&ctl.s_empty));
+          // the peer's buffer gt & 1 is free once its copy of tile gt - 1 left it
+          if (lane == 0) {
+            const uint32_t par = ((((gt + 1) >> 1) - 1u) & 1u);
+            ok = mbar_wait<true>(smem_u32(&ctl.tx_ok[warp][gt & 1]), par, abort, timeout_ns);
           }
-          tmem_wait_st();
-        }
-        if (grow_max) {
-          l_run *= alpha;
-          m_run = mt;
-        }
-        uint32_t pk[32];
-        float psum = 0.f;
-        const bool any = m_run != -INFINITY;
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          const uint32_t stage_off = chunk_off + ((gt + 1) & 1) * kXBytes;   // outgoing: buffer (gt + 1) & 1
 #pragma unroll
-        for (int k = 0; k < 64; k += 2) {
-          const float p0 = any ? ex2_approx(x[k] - m_run) : 0.f;
-          const float p1 = any ? ex2_approx(x[k + 1] - m_run) : 0.f;
-          psum += p0 + p1;
-          pk[k >> 1] = pack_bf16x2(p0, p1);
-        }
-        l_run += psum;
-        const uint32_t tp = tmem + lane_off + kTmemP + 32 * sb;
-        tmem_st16(tp, pk);
-        tmem_st16(tp + 16, pk + 16);
-        tmem_wait_st();
-
-        // Slots past the sequence end in its last block may hold anything (NaN): zero
-        // those token rows of this CTA's latent slice before the PV reads them.
-        const int tail = sg.Lc % kBS;
-        if (tile == last_tile && tail != 0) {
-          const uint32_t st = g % kStages;
-          int dummy = 0;
-          mbar_wait<false>(smem_u32(&ctl.kv_full[st]), (g / kStages) & 1, &dummy, timeout_ns);
-          uint8_t* base = smem + kOffKv + st * kStageBytes;
-          const int pieces = 4 * (kBS - tail) * 8;        // 16-byte pieces
-          for (int i = row; i < pieces; i += 128) {
-            const int chunk = i / ((kBS - tail) * 8);
-            const int rem = i % ((kBS - tail) * 8);
-            const int tok = tail + rem / 8;
-            *reinterpret_cast<uint4*>(base + chunk * kKvLatChunk + tok * 128 + (rem % 8) * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-          }
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(smem + stage_off + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3]);
           fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            bulk_copy_to_peer(peer_x0 + (gt & 1) * kXBytes, smem_u32(smem + kOffX + ((gt + 1) & 1) * kXBytes +
+                                                                        warp * kXChunk),
+                              kXChunk, (gt & 1) ? peer_rx_full1 : peer_rx_full0);
+            bulk_commit_group();
+          }
         }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&ctl.p_full[sb]));
+        if (li > 0) {
+          // ---- B2: exponentials of tile gt - 1, P into TMEM
+          const uint32_t gp = gt - 1;
+          const int tile = sg.tile_begin + li - 1;
+          const bool grow_max = mt > m_run + kRescaleThreshold;
+          const bool rescale = grow_max && m_run != -INFINITY;
+          const float alpha = rescale ? ex2_approx(m_run - mt) : 1.f;
+          if (__any_sync(0xffffffffu, rescale)) {
+            // O holds this segment's tiles before gp: wait for their last two PVs (older
+            // ones are known complete), then scale in place
+            ok = (gp < g + 2 || wait_pv(gp - 2)) && wait_pv(gp - 1);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+              uint32_t v[16];
+              const uint32_t ta = tmem + lane_off + kTmemO + 128 * half + 16 * c;
+              tmem_ld16(ta, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+              tmem_st16(ta, v);
+            }
+            tmem_wait_st();
+          }
+          if (grow_max) {
+            l_run *= alpha;
+            m_run = mt;
+          }
+          uint32_t pk[16];
+          float psum = 0.f;
+          const bool any = m_run != -INFINITY;
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const float p0 = any ? ex2_approx(x[k] - m_run) : 0.f;
+            const float p1 = any ? ex2_approx(x[k + 1] - m_run) : 0.f;
+            psum += p0 + p1;
+            pk[k >> 1] = pack_bf16x2(p0, p1);
+          }
+          l_run += psum;
+          tmem_st16(tmem + lane_off + kTmemP + 32 * (gp & 1) + 16 * half, pk);
+          tmem_wait_st();
+          // Slots past the sequence end in its last block may hold anything (NaN): zero
+          // those token rows of this CTA's latent slice before the PV reads them.
+          const int tail = sg.Lc % kBS;
+          if (tile == last_tile && tail != 0) {
+            const uint32_t stg = gp % kStages;
+            int dummy = 0;
+            mbar_wait<false>(smem_u32(&ctl.kv_full[stg]), (gp / kStages) & 1, &dummy, timeout_ns);
+            uint8_t* base = smem + kOffKv + stg * kStageBytes;
+            const int per_chunk = (kBS - tail) * 8;          // 16-byte pieces per chunk
+            for (int i = st_idx; i < 4 * per_chunk; i += kSoftmaxThreads) {
+              const int chunk = i / per_chunk, rem = i % per_chunk;
+              *reinterpret_cast<uint4*>(base + chunk * kKvLatChunk + (tail + rem / 8) * 128 + (rem % 8) * 16) =
+                  make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();
+          }
+          tc_fence_before();
+          mbar_arrive(smem_u32(&ctl.p_full[gp & 1]));
+        }
+        if (li < n) {
+          // ---- B1: the peer's partials of tile gt; full scores; row maximum
+          const int tile = sg.tile_begin + li;
+          if (lane == 0) {
+            // our outgoing copy no longer reads buffer (gt + 1) & 1: the peer may fill it
+            bulk_wait_group_read<0>();
+            mbar_arrive_remote(((gt + 1) & 1) ? peer_tx_ok1 : peer_tx_ok0);
+          }
+          ok = wait_peer(smem_u32(&ctl.rx_full[gt & 1]), (gt >> 1) & 1);
+          if (!ok) break;
+          if (st_idx == 0) mbar_arrive_expect_tx(smem_u32(&ctl.rx_full[gt & 1]), kXBytes);   // tile gt + 2
+          const uint32_t in_off = chunk_off + (gt & 1) * kXBytes;
+          const int valid = min(max(n_row - tile * kBS - 32 * half, 0), 32);   // of my 32 columns
+          float mh = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(smem + in_off + ((c ^ (lane & 7)) << 4));
+            const float r4[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                                 __uint_as_float(v.w)};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int k = 4 * c + i;
+              const float sc = (__uint_as_float(sv[k]) + r4[i]) * scale_log2;
+              x[k] = k < valid ? sc : -INFINITY;
+              mh = fmaxf(mh, x[k]);
+            }
+          }
+          ctl.mbuf[gt & 1][half][row] = mh;
+          mbar_arrive(smem_u32(&ctl.mx[quad]));
+          ok = wait_local(smem_u32(&ctl.mx[quad]), gt & 1);
+          if (!ok) break;
+          mt = fmaxf(ctl.mbuf[gt & 1][0][row], ctl.mbuf[gt & 1][1][row]);
+        }
       }
       if (!ok) break;
+      g += n;
 
       // epilogue: O / l -> out (single split) or the normalised partial (several splits).
-      // Only the PV before the last tile's QK is known complete, and a parity wait only
-      // tells the last two phases apart: wait for the second-to-last PV, then the last.
-      const uint32_t gl = g - 1;
-      ok = (gl == 0 || wait_local(smem_u32(&ctl.pv_done), (gl - 1) & 1)) &&
-           wait_local(smem_u32(&ctl.pv_done), gl & 1);
+      // Known complete: the PV three tiles before the last; wait for the last three PVs
+      // of this segment in order.
+      for (uint32_t j = (n >= 3 ? g - 3 : g - n); ok && j < g; ++j) ok = wait_pv(j);
       if (!ok) break;
       tc_fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      const float lse_v = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      ctl.lbuf[half][row] = l_run;
+      mbar_arrive(smem_u32(&ctl.lx[quad]));
+      ok = wait_local(smem_u32(&ctl.lx[quad]), seg & 1);
+      if (!ok) break;
+      const float l_tot = ctl.lbuf[0][row] + ctl.lbuf[1][row];
+      const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      const float lse_v = l_tot > 0.f ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
       const size_t qrow = (size_t)sg.b * a.rows + grow;
       const bool direct = sg.splits == 1;
       const size_t prow = (size_t)(w + sg.b) * a.rows + grow;
 #pragma unroll 1
-      for (int c = 0; c < 16; ++c) {
+      for (int c = 0; c < 8; ++c) {
         uint32_t v[16];
-        tmem_ld16(tmem + lane_off + kTmemO + 16 * c, v);
+        tmem_ld16(tmem + lane_off + kTmemO + 128 * half + 16 * c, v);
         tmem_wait_ld();
         if (!valid_row) continue;
-        const int ch = 256 * (int)rank + 16 * c;
+        const int ch = 256 * (int)rank + 128 * half + 16 * c;
         if (direct && a.out_dtype == kBF16) {
           uint4 o0, o1;
           o0.x = pack_bf16x2(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv);
@@ -433,18 +512,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             __uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
         }
       }
-      if (valid_row && rank == 0) {
+      if (valid_row && rank == 0 && half == 0) {
         if (direct)
           a.lse[qrow] = lse_v;
         else
           a.lse_part[prow] = lse_v;
       }
-      if (sg.split == 0 && rg == 0 && rank == 0 && row == 0) {
+      if (sg.split == 0 && rg == 0 && rank == 0 && st_idx == 0) {
         a.meta[2 * sg.b] = sg.first_worker;
         a.meta[2 * sg.b + 1] = sg.splits;
       }
       tc_fence_before();
+      ++seg;
     }
+    if (lane == 0) bulk_wait_group_read<0>();
     if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
   }
 
@@ -508,10 +589,9 @@ bool tc_workers_ok(int W, int rows) { return W >= 1 && (long long)W * row_groups
 
 cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
   const int n_rg = row_groups(a.rows);
-  CUtensorMap tq, tqr, tkv, tkr;
+  CUtensorMap tqr, tkv, tkr;
   const uint64_t rows = (uint64_t)a.rows;
-  if (!make_map_3d(&tq, a.q_lat, kR, rows, a.B, kR * 2, rows * kR * 2, 64, kRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_3d(&tqr, a.q_rope, kDR, rows, a.B, kDR * 2, rows * kDR * 2, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B) ||
+  if (!make_map_3d(&tqr, a.q_rope, kDR, rows, a.B, kDR * 2, rows * kDR * 2, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_map_3d(&tkv, a.cache, kR + kDR, kBS, a.num_blocks, (kR + kDR) * 2, (uint64_t)kBS * (kR + kDR) * 2, 64,
                    kBS, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_3d(&tkr, a.cache, kR + kDR, kBS, a.num_blocks, (kR + kDR) * 2, (uint64_t)kBS * (kR + kDR) * 2, 32,
@@ -527,7 +607,7 @@ cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
   if (attr_err != cudaSuccess) return attr_err;
   const uint64_t timeout_ns = 2000000000ull;
   const dim3 grid(2 * a.W * n_rg);
-  tc_decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tqr, tkv, tkr, a, n_rg, timeout_ns);
+  tc_decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(tqr, tkv, tkr, a, n_rg, timeout_ns);
   return cudaGetLastError();
 }
 
