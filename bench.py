@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller profiling captures only)")
     return ap.parse_args()
 
 
@@ -209,6 +211,9 @@ def main():
 
     import head_latent_attention_split_b200 as mla
     wl = W.BY_NAME[args.workload]
+    if args.batch is not None and args.batch != wl.B:
+        lens = wl.seq_lens if isinstance(wl.seq_lens, str) else tuple(wl.seq_lens[:1]) * args.batch
+        wl = wl.with_(B=args.batch, seq_lens=lens, name=f"{wl.name}_b{args.batch}")
     inp = W.make_inputs(wl, threads=max(1, (os.cpu_count() or 1) // world))
     t = W.to_torch(inp, f"cuda:{local}")
     p = mla.params_for(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], wl.scale, wl.causal,
@@ -287,7 +292,7 @@ def main():
     h2d = sum(x.numel() * x.element_size() for x in (hq, hqr, hbt, hsl))
     d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
     e2e_ms = 0.0
-    for i in range(E + 2):
+    for i in range(E + 2 if E > 0 else 0):
         if flush:
             flush_buf.fill_(1.0)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -346,7 +351,7 @@ def main():
                 peaks=peaks),
             cpu_baseline=cpu,
             e2e=dict(value=world * E * model["cache_bytes"] / (e2e_ms / 1e3) / 1e12, unit="TB/s",
-                     h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms / E),
+                     h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms / E) if E > 0 else None,
             gpu_launches=2 * K,
             clocks=clocks,
         )

@@ -1,5 +1,5 @@
 // Tensor-core (tcgen05 + TMA) absorbed-MLA decode for r = 512, d_r = 64, 64-token
-// cache blocks, bf16 queries, bf16 cache.
+// cache blocks, bf16 queries, bf16 or FP8 e4m3 (per-token scale) cache.
 //
 // Design (one CTA pair = one cluster of 2 per worker and row group):
 //  * The 128 query rows of a row group (Sq * H rows of one sequence, zero-padded) are
@@ -31,11 +31,21 @@
 //  * PV: O_j[128 x 256] += P[128 x 64] . C_j[64 x 256] with A = P from TMEM and B =
 //    the SAME shared-memory tile the QK used, read N-major (4 MMAs, N = 256). The MMA
 //    issuer runs QK(k) then PV(k - 2).
+//  * FP8 cache, exact: c_t = code_t * s_t with a per-token fp32 scale s_t. The
+//    producer TMA-loads the CTA's 256 e4m3 codes per token (16 KB) into the upper half
+//    of the stage and the bf16 RoPE key into its slot; two converter warps (one token row
+//    per thread) write the codes back as bf16 in place (every e4m3 value is exact in
+//    bf16) in the 128B-swizzled layout the bf16 path loads, and replace the RoPE key by
+//    kR_t / s_t split into bf16 hi + lo parts (2^-16 relative). The score MMAs then give
+//    S_t / s_t; the softmax multiplies each column by s_t, and P by s_t before PV
+//    (sum_t p_t s_t code_t = sum_t p_t c_t), with the row sum over the unscaled p_t.
 //  * Warp roles: warps 0-7 softmax / epilogue, warp 8 TMA producer, warp 9 TMEM
-//    allocator and single-thread MMA issuer; mbarrier pipelines between them. Every
-//    wait is bounded (timeout -> MLA_ERR_TIMEOUT, clean exit).
+//    allocator and single-thread MMA issuer, warps 10-11 FP8 converters; mbarrier
+//    pipelines between them. Every wait is bounded (timeout -> MLA_ERR_TIMEOUT,
+//    clean exit).
 // The work split over workers (CTA pairs) is the flat block list plan of mla_device.cuh.
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include <cmath>
 #include <mutex>
@@ -51,17 +61,25 @@ using namespace ptx;
 
 constexpr int kR = 512, kDR = 64, kBS = 64;
 constexpr int kRows = 128;           // query rows per row group = MMA M
-constexpr int kStages = 4;
+constexpr int kMaxStages = 4;
 
 // shared memory layout, byte offsets from a 1024-aligned base
 constexpr uint32_t kKvLatChunk = kBS * 128;                      // [64 tok][64 ch] bf16, 128B swizzle
 constexpr uint32_t kKvRope = kBS * 64;                           // [64 tok][32 ch] bf16, 64B swizzle
-constexpr uint32_t kStageBytes = 4 * kKvLatChunk + kKvRope;      // 36864
+// bf16 stage: latent chunks + RoPE. FP8 stage: latent chunks + RoPE hi + RoPE lo + scales.
+template <bool kFp8> struct Geo {
+  static constexpr int kStages = kFp8 ? 3 : 4;
+  static constexpr uint32_t kStageBytes = kFp8 ? 41984u : 36864u;
+  static constexpr uint32_t kOffRopeLo = 4 * kKvLatChunk + kKvRope;   // FP8 only
+  static constexpr uint32_t kOffScale = kOffRopeLo + kKvRope;         // FP8 only: 64 fp32
+};
+static_assert(Geo<true>::kOffScale + 256 <= Geo<true>::kStageBytes && Geo<true>::kStageBytes % 1024 == 0, "fp8 stage");
 constexpr uint32_t kQRope = kRows * 64;                          // [128 rows][32 ch] bf16, 64B swizzle
 constexpr uint32_t kXBytes = kRows * 64 * 4;                     // partial scores [128 rows][64] fp32
 constexpr uint32_t kXChunk = kXBytes / 8;                        // one softmax warp's 32 rows x 32 cols
 constexpr uint32_t kOffKv = 0;
-constexpr uint32_t kOffQr = kOffKv + kStages * kStageBytes;
+constexpr uint32_t kOffQr = 4 * 36864;   // after the stages (both cache types use <= 147456 bytes)
+static_assert(Geo<true>::kStages * Geo<true>::kStageBytes <= kOffQr, "stages fit");
 constexpr uint32_t kOffX = kOffQr + kQRope;                      // two exchange buffers
 constexpr uint32_t kOffCtl = kOffX + 2 * kXBytes;
 constexpr uint32_t kCtlBytes = 4096;
@@ -79,13 +97,18 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kSoftmaxThreads = 256;  // warps 0-7
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kConvWarp0 = 10;        // FP8 cache only: warps 10-11 decode codes in place
+constexpr int kConvThreads = 64;      // one thread per token row of a tile
+template <bool kFp8>
+constexpr int threads_for() { return kFp8 ? 384 : 320; }
+constexpr uint32_t kFp8CodeBytes = kBS * 256;                    // this CTA's codes of one block
+constexpr uint32_t kFp8StageTx = kFp8CodeBytes + kKvRope;
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only if the max grows > 2^8
 
 struct Ctl {
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
+  uint64_t kv_full[kMaxStages];
+  uint64_t kv_empty[kMaxStages];
   uint64_t q_full, q_empty;
   uint64_t s_full, s_empty;
   uint64_t p_full[2];
@@ -94,6 +117,8 @@ struct Ctl {
   uint64_t tx_ok[8][2];     // per warp: the peer's buffer b may take our next partials
   uint64_t mx[4];           // the two warps sharing 32 rows published their tile maxima
   uint64_t lx[4];           // ... their row sums
+  uint64_t kv_ready[kMaxStages];   // FP8: the converted bf16 tile is in place
+  uint64_t cv_loaded[kMaxStages];  // FP8: every converter thread holds its codes in registers
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -109,10 +134,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// e4m3 pair (low byte = first code) -> two fp32, exact (hardware cvt to f16x2 first)
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two_codes) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(h2) : "r"(two_codes));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
+}
+
+template <bool kFp8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(), 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_kr, const DecodeArgs a, const int n_rg,
                      const uint64_t timeout_ns) {
+  constexpr int kStages = Geo<kFp8>::kStages;
+  constexpr uint32_t kStageBytes = Geo<kFp8>::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   Ctl& ctl = *reinterpret_cast<Ctl*>(smem + kOffCtl);
@@ -146,6 +181,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 4; ++i) {
       mbar_init(smem_u32(&ctl.mx[i]), 64);
       mbar_init(smem_u32(&ctl.lx[i]), 64);
+    }
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(smem_u32(&ctl.kv_ready[i]), kConvThreads);
+      mbar_init(smem_u32(&ctl.cv_loaded[i]), kConvThreads);
     }
     mbar_init(smem_u32(&ctl.drain), 1);
     ctl.abort = 0;
@@ -190,9 +229,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int blk = checked_block(a.block_table, a.max_blocks, sg.b, tile, a.num_blocks, a.status);
           const uint32_t bar = smem_u32(&ctl.kv_full[st]);
           const uint32_t base = sKv + st * kStageBytes;
-          mbar_arrive_expect_tx(bar, kStageBytes);
-          for (int c = 0; c < 4; ++c) tma_load_3d(base + c * kKvLatChunk, &tm_kv, bar, 256 * rank + 64 * c, 0, blk);
-          tma_load_3d(base + 4 * kKvLatChunk, &tm_kr, bar, kR + 32 * rank, 0, blk);
+          if constexpr (kFp8) {
+            // codes [64 tok][256 B] into the upper half of the latent area, RoPE key into its slot
+            mbar_arrive_expect_tx(bar, kFp8StageTx);
+            tma_load_3d(base + 2 * kKvLatChunk, &tm_kv, bar, 256 * rank, 0, blk);
+            tma_load_3d(base + 4 * kKvLatChunk, &tm_kr, bar, 32 * rank, 0, blk);
+          } else {
+            mbar_arrive_expect_tx(bar, kStageBytes);
+            for (int c = 0; c < 4; ++c) tma_load_3d(base + c * kKvLatChunk, &tm_kv, bar, 256 * rank + 64 * c, 0, blk);
+            tma_load_3d(base + 4 * kKvLatChunk, &tm_kr, bar, kR + 32 * rank, 0, blk);
+          }
         }
         ++seg;
       }
@@ -237,7 +283,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int n = sg.tile_end - sg.tile_begin;
         for (int li = 0; li < n; ++li, ++g) {
           const uint32_t st = g % kStages;
-          ok = mbar_wait<false>(smem_u32(&ctl.kv_full[st]), (g / kStages) & 1, abort, timeout_ns) &&
+          ok = mbar_wait<false>(smem_u32(kFp8 ? &ctl.kv_ready[st] : &ctl.kv_full[st]), (g / kStages) & 1, abort,
+                                timeout_ns) &&
                mbar_wait<false>(smem_u32(&ctl.s_empty), (g & 1) ^ 1, abort, timeout_ns);
           if (!ok) break;
           tc_fence_after();
@@ -250,9 +297,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mma_ts(d, tmem + kTmemQ + 8 * kk, bdesc, idesc_qk, kk ? 1u : 0u);
           }
 #pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            const uint64_t adesc = smem_desc(sQr + kk * 32, 16, 512, kSwizzle64B);
-            const uint64_t bdesc = smem_desc(base + 4 * kKvLatChunk + kk * 32, 16, 512, kSwizzle64B);
+          for (int kk = 0; kk < (kFp8 ? 4 : 2); ++kk) {
+            // RoPE channels; FP8: k-steps 2, 3 repeat the query against the lo parts
+            const uint64_t adesc = smem_desc(sQr + (kk & 1) * 32, 16, 512, kSwizzle64B);
+            const uint64_t bdesc =
+                smem_desc(base + (kk < 2 ? 4 * kKvLatChunk : Geo<kFp8>::kOffRopeLo) + (kk & 1) * 32, 16, 512,
+                          kSwizzle64B);
             mma_ss(d, adesc, bdesc, idesc_qk, 1u);
           }
           mma_commit(smem_u32(&ctl.s_full));
@@ -270,6 +320,87 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int dummy = 0;
       mma_commit(smem_u32(&ctl.drain));
       mbar_wait<false>(smem_u32(&ctl.drain), 0, &dummy, timeout_ns);
+      if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
+    }
+  } else if (warp >= kConvWarp0) {
+    // ------------------------------------------------------------------ FP8 converters
+    if constexpr (kFp8) {
+      const int tok = threadIdx.x - kConvWarp0 * 32;     // token row of the tile, 0..63
+      SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
+      Segment sg;
+      uint32_t g = 0;
+      bool ok = true;
+      while (ok && it.next(sg)) {
+        for (int tile = sg.tile_begin; tile < sg.tile_end; ++tile, ++g) {
+          const uint32_t st = g % kStages, ph = (g / kStages) & 1;
+          ok = __all_sync(0xffffffffu, mbar_wait<false>(smem_u32(&ctl.kv_full[st]), ph, abort, timeout_ns));
+          if (!ok) break;
+          const int blk = checked_block(a.block_table, a.max_blocks, sg.b, tile, a.num_blocks, a.status);
+          const float sc = __ldg(a.kv_scale + (size_t)blk * kBS + tok);
+          uint8_t* base = smem + kOffKv + st * kStageBytes;
+          // RoPE key / scale as bf16 hi + lo (its 64-byte row, 64B-swizzled, in place + lo slot)
+          {
+            const float inv_sc = 1.0f / sc;
+            uint8_t* hi_row = base + 4 * kKvLatChunk + tok * 64;
+            uint8_t* lo_row = base + Geo<kFp8>::kOffRopeLo + tok * 64;
+#pragma unroll
+            for (int pc = 0; pc < 4; ++pc) {
+              const int phys = (pc ^ ((tok >> 1) & 3)) << 4;
+              const uint4 v = *reinterpret_cast<const uint4*>(hi_row + phys);
+              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+              uint32_t h[4], l[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float x0 = __uint_as_float(wv[j] << 16) * inv_sc;
+                const float x1 = __uint_as_float(wv[j] & 0xFFFF0000u) * inv_sc;
+                h[j] = pack_bf16x2(x0, x1);
+                l[j] = pack_bf16x2(x0 - __uint_as_float(h[j] << 16), x1 - __uint_as_float(h[j] & 0xFFFF0000u));
+              }
+              *reinterpret_cast<uint4*>(hi_row + phys) = make_uint4(h[0], h[1], h[2], h[3]);
+              *reinterpret_cast<uint4*>(lo_row + phys) = make_uint4(l[0], l[1], l[2], l[3]);
+            }
+            *reinterpret_cast<float*>(base + Geo<kFp8>::kOffScale + tok * 4) = sc;
+          }
+          // codes of this token: 16 pieces of 16 bytes (channels [16 p, 16 p + 16)). Piece
+          // order is XOR-staggered by the token so that a warp's loads hit distinct banks.
+          const uint8_t* src = base + 2 * kKvLatChunk + tok * 256;
+          auto convert_piece = [&](const uint4 v, const int p) {
+            // -> channels [16 p, 16 p + 16): chunk p / 4, 16-byte pieces 2 (p % 4) and
+            // 2 (p % 4) + 1 of the 128B-swizzled row
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 lo = e4m3x2_to_float2(wv[j] & 0xFFFFu);
+              const float2 hi = e4m3x2_to_float2(wv[j] >> 16);
+              o[2 * j] = pack_bf16x2(lo.x, lo.y);            // exact: e4m3 values fit bf16
+              o[2 * j + 1] = pack_bf16x2(hi.x, hi.y);
+            }
+            uint8_t* row = base + (p >> 2) * kKvLatChunk + tok * 128;
+            const int p0 = 2 * (p & 3);
+            *reinterpret_cast<uint4*>(row + (((p0) ^ (tok & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(row + (((p0 + 1) ^ (tok & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+          };
+          // pieces 8-15 live where chunks 2-3 will be written: hold them in registers
+          uint4 upper[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) upper[j] = *reinterpret_cast<const uint4*>(src + ((8 + (j ^ (tok & 7))) << 4));
+          // pieces 0-7 convert straight into chunks 0-1 (which hold no codes)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int pc = j ^ (tok & 7);
+            convert_piece(*reinterpret_cast<const uint4*>(src + (pc << 4)), pc);
+          }
+          // every row's upper codes are in registers before any row's bf16 lands on them
+          mbar_arrive(smem_u32(&ctl.cv_loaded[st]));
+          ok = __all_sync(0xffffffffu, mbar_wait<false>(smem_u32(&ctl.cv_loaded[st]), ph, abort, timeout_ns));
+          if (!ok) break;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) convert_piece(upper[j], 8 + (j ^ (tok & 7)));
+          fence_proxy_async_smem();
+          mbar_arrive(smem_u32(&ctl.kv_ready[st]));
+        }
+      }
       if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
     }
   } else {
@@ -401,12 +532,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
           float psum = 0.f;
           const bool any = m_run != -INFINITY;
+          float pcs[32];     // FP8: P columns carry the token scale into PV (0 for unseen tokens)
+          if constexpr (kFp8) {
+            const int valid_p = min(max(n_row - tile * kBS - 32 * half, 0), 32);
+            const float4* cs = reinterpret_cast<const float4*>(smem + kOffKv + (gp % kStages) * kStageBytes +
+                                                               Geo<kFp8>::kOffScale + 128 * half);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float4 v = cs[c];
+              pcs[4 * c] = 4 * c < valid_p ? v.x : 0.f;
+              pcs[4 * c + 1] = 4 * c + 1 < valid_p ? v.y : 0.f;
+              pcs[4 * c + 2] = 4 * c + 2 < valid_p ? v.z : 0.f;
+              pcs[4 * c + 3] = 4 * c + 3 < valid_p ? v.w : 0.f;
+            }
+          }
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
             const float p0 = any ? ex2_approx(x[k] - m_run) : 0.f;
             const float p1 = any ? ex2_approx(x[k + 1] - m_run) : 0.f;
             psum += p0 + p1;
-            pk[k >> 1] = pack_bf16x2(p0, p1);
+            if constexpr (kFp8)
+              pk[k >> 1] = pack_bf16x2(p0 * pcs[k], p1 * pcs[k + 1]);
+            else
+              pk[k >> 1] = pack_bf16x2(p0, p1);
           }
           l_run += psum;
           tmem_st16(tmem + lane_off + kTmemP + 32 * (gp & 1) + 16 * half, pk);
@@ -417,7 +565,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (tile == last_tile && tail != 0) {
             const uint32_t stg = gp % kStages;
             int dummy = 0;
-            mbar_wait<false>(smem_u32(&ctl.kv_full[stg]), (gp / kStages) & 1, &dummy, timeout_ns);
+            mbar_wait<false>(smem_u32(kFp8 ? &ctl.kv_ready[stg] : &ctl.kv_full[stg]), (gp / kStages) & 1, &dummy,
+                             timeout_ns);
             uint8_t* base = smem + kOffKv + stg * kStageBytes;
             const int per_chunk = (kBS - tail) * 8;          // 16-byte pieces per chunk
             for (int i = st_idx; i < 4 * per_chunk; i += kSoftmaxThreads) {
@@ -443,6 +592,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (st_idx == 0) mbar_arrive_expect_tx(smem_u32(&ctl.rx_full[gt & 1]), kXBytes);   // tile gt + 2
           const uint32_t in_off = chunk_off + (gt & 1) * kXBytes;
           const int valid = min(max(n_row - tile * kBS - 32 * half, 0), 32);   // of my 32 columns
+          float colsc[32];   // FP8: token scales of my columns (1 for the bf16 cache)
+          if constexpr (kFp8) {
+            const uint32_t stg = gt % kStages;
+            int dummy = 0;
+            mbar_wait<false>(smem_u32(&ctl.kv_ready[stg]), (gt / kStages) & 1, &dummy, timeout_ns);
+            const float4* cs = reinterpret_cast<const float4*>(smem + kOffKv + stg * kStageBytes +
+                                                               Geo<kFp8>::kOffScale + 128 * half);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float4 v = cs[c];
+              colsc[4 * c] = v.x;
+              colsc[4 * c + 1] = v.y;
+              colsc[4 * c + 2] = v.z;
+              colsc[4 * c + 3] = v.w;
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) colsc[k] = 1.f;
+          }
           float mh = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -452,7 +620,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int k = 4 * c + i;
-              const float sc = (__uint_as_float(sv[k]) + r4[i]) * scale_log2;
+              const float sc = (__uint_as_float(sv[k]) + r4[i]) * colsc[k] * scale_log2;
               x[k] = k < valid ? sc : -INFINITY;
               mh = fmaxf(mh, x[k]);
             }
@@ -557,16 +725,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D bf16 tensor map: dims (inner -> outer), byte strides of dims 1 and 2, box.
+// 3-D tensor map: dims (inner -> outer), byte strides of dims 1 and 2, box.
 bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
-                 uint64_t s2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+                 uint64_t s2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw,
+                 CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
   const cuuint64_t strides[2] = {s1, s2};
   const cuuint32_t box[3] = {b0, b1, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -576,7 +745,8 @@ int row_groups(int rows) { return (rows + kRows - 1) / kRows; }
 }  // namespace
 
 bool tc_supported(int r, int d_r, int block_size, int q_dtype, int cache_dtype, int out_dtype, int rows) {
-  return r == kR && d_r == kDR && block_size == kBS && q_dtype == kBF16 && cache_dtype == kBF16 &&
+  return r == kR && d_r == kDR && block_size == kBS && q_dtype == kBF16 &&
+         (cache_dtype == kBF16 || cache_dtype == kE4M3) &&
          (out_dtype == kBF16 || out_dtype == kF32) && rows >= 1 && row_groups(rows) <= 1024;
 }
 
@@ -591,23 +761,40 @@ cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
   const int n_rg = row_groups(a.rows);
   CUtensorMap tqr, tkv, tkr;
   const uint64_t rows = (uint64_t)a.rows;
-  if (!make_map_3d(&tqr, a.q_rope, kDR, rows, a.B, kDR * 2, rows * kDR * 2, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map_3d(&tkv, a.cache, kR + kDR, kBS, a.num_blocks, (kR + kDR) * 2, (uint64_t)kBS * (kR + kDR) * 2, 64,
-                   kBS, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_3d(&tkr, a.cache, kR + kDR, kBS, a.num_blocks, (kR + kDR) * 2, (uint64_t)kBS * (kR + kDR) * 2, 32,
-                   kBS, CU_TENSOR_MAP_SWIZZLE_64B))
-    return cudaErrorInvalidValue;
-  static std::once_flag attr_once[64];
+  const bool fp8 = a.cache_dtype == kE4M3;
+  bool ok = make_map_3d(&tqr, a.q_rope, kDR, rows, a.B, kDR * 2, rows * kDR * 2, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (fp8) {
+    // codes [num_blocks][64][512] e4m3 (256-byte boxes, no swizzle), RoPE keys [num_blocks][64][64] bf16
+    ok = ok &&
+         make_map_3d(&tkv, a.cache, kR, kBS, a.num_blocks, kR, (uint64_t)kBS * kR, 256, kBS, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_DATA_TYPE_UINT8) &&
+         make_map_3d(&tkr, a.k_rope, kDR, kBS, a.num_blocks, kDR * 2, (uint64_t)kBS * kDR * 2, 32, kBS,
+                     CU_TENSOR_MAP_SWIZZLE_64B);
+  } else {
+    ok = ok &&
+         make_map_3d(&tkv, a.cache, kR + kDR, kBS, a.num_blocks, (kR + kDR) * 2, (uint64_t)kBS * (kR + kDR) * 2, 64,
+                     kBS, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map_3d(&tkr, a.cache, kR + kDR, kBS, a.num_blocks, (kR + kDR) * 2, (uint64_t)kBS * (kR + kDR) * 2, 32,
+                     kBS, CU_TENSOR_MAP_SWIZZLE_64B);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  static std::once_flag attr_once[2][64];
   int dev = 0;
   cudaGetDevice(&dev);
   cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once[dev & 63], [&] {
-    attr_err = cudaFuncSetAttribute(tc_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  std::call_once(attr_once[fp8 ? 1 : 0][dev & 63], [&] {
+    attr_err = fp8 ? cudaFuncSetAttribute(tc_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          kSmemBytes)
+                   : cudaFuncSetAttribute(tc_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
   const uint64_t timeout_ns = 2000000000ull;
   const dim3 grid(2 * a.W * n_rg);
-  tc_decode_kernel<<<grid, kThreads, kSmemBytes, s>>>(tqr, tkv, tkr, a, n_rg, timeout_ns);
+  if (fp8)
+    tc_decode_kernel<true><<<grid, threads_for<true>(), kSmemBytes, s>>>(tqr, tkv, tkr, a, n_rg, timeout_ns);
+  else
+    tc_decode_kernel<false><<<grid, threads_for<false>(), kSmemBytes, s>>>(tqr, tkv, tkr, a, n_rg, timeout_ns);
   return cudaGetLastError();
 }
 
