@@ -102,7 +102,7 @@ constexpr int kConvThreads = 64;      // one thread per token row of a tile
 template <bool kFp8>
 constexpr int threads_for() { return kFp8 ? 384 : 320; }
 constexpr uint32_t kFp8CodeBytes = kBS * 256;                    // this CTA's codes of one block
-constexpr uint32_t kFp8StageTx = kFp8CodeBytes + kKvRope;
+constexpr uint32_t kFp8StageTx = kFp8CodeBytes + kKvRope + kBS * 4;   // codes, RoPE key, scales
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only if the max grows > 2^8
 
@@ -144,8 +144,8 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two_codes) {
 template <bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(), 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_kv,
-                     const __grid_constant__ CUtensorMap tm_kr, const DecodeArgs a, const int n_rg,
-                     const uint64_t timeout_ns) {
+                     const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_sc,
+                     const DecodeArgs a, const int n_rg, const uint64_t timeout_ns) {
   constexpr int kStages = Geo<kFp8>::kStages;
   constexpr uint32_t kStageBytes = Geo<kFp8>::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
@@ -234,6 +234,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
             mbar_arrive_expect_tx(bar, kFp8StageTx);
             tma_load_3d(base + 2 * kKvLatChunk, &tm_kv, bar, 256 * rank, 0, blk);
             tma_load_3d(base + 4 * kKvLatChunk, &tm_kr, bar, 32 * rank, 0, blk);
+            tma_load_3d(base + Geo<kFp8>::kOffScale, &tm_sc, bar, 0, 0, blk);
           } else {
             mbar_arrive_expect_tx(bar, kStageBytes);
             for (int c = 0; c < 4; ++c) tma_load_3d(base + c * kKvLatChunk, &tm_kv, bar, 256 * rank + 64 * c, 0, blk);
@@ -335,9 +336,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
           const uint32_t st = g % kStages, ph = (g / kStages) & 1;
           ok = __all_sync(0xffffffffu, mbar_wait<false>(smem_u32(&ctl.kv_full[st]), ph, abort, timeout_ns));
           if (!ok) break;
-          const int blk = checked_block(a.block_table, a.max_blocks, sg.b, tile, a.num_blocks, a.status);
-          const float sc = __ldg(a.kv_scale + (size_t)blk * kBS + tok);
           uint8_t* base = smem + kOffKv + st * kStageBytes;
+          const float sc = *reinterpret_cast<const float*>(base + Geo<kFp8>::kOffScale + tok * 4);   // TMA'd
           // RoPE key / scale as bf16 hi + lo (its 64-byte row, 64B-swizzled, in place + lo slot)
           {
             const float inv_sc = 1.0f / sc;
@@ -359,7 +359,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
               *reinterpret_cast<uint4*>(hi_row + phys) = make_uint4(h[0], h[1], h[2], h[3]);
               *reinterpret_cast<uint4*>(lo_row + phys) = make_uint4(l[0], l[1], l[2], l[3]);
             }
-            *reinterpret_cast<float*>(base + Geo<kFp8>::kOffScale + tok * 4) = sc;
           }
           // codes of this token: 16 pieces of 16 bytes (channels [16 p, 16 p + 16)). Piece
           // order is XOR-staggered by the token so that a warp's loads hit distinct banks.
@@ -759,7 +758,7 @@ bool tc_workers_ok(int W, int rows) { return W >= 1 && (long long)W * row_groups
 
 cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
   const int n_rg = row_groups(a.rows);
-  CUtensorMap tqr, tkv, tkr;
+  CUtensorMap tqr, tkv, tkr, tsc;
   const uint64_t rows = (uint64_t)a.rows;
   const bool fp8 = a.cache_dtype == kE4M3;
   bool ok = make_map_3d(&tqr, a.q_rope, kDR, rows, a.B, kDR * 2, rows * kDR * 2, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B);
@@ -769,7 +768,9 @@ cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
          make_map_3d(&tkv, a.cache, kR, kBS, a.num_blocks, kR, (uint64_t)kBS * kR, 256, kBS, CU_TENSOR_MAP_SWIZZLE_NONE,
                      CU_TENSOR_MAP_DATA_TYPE_UINT8) &&
          make_map_3d(&tkr, a.k_rope, kDR, kBS, a.num_blocks, kDR * 2, (uint64_t)kBS * kDR * 2, 32, kBS,
-                     CU_TENSOR_MAP_SWIZZLE_64B);
+                     CU_TENSOR_MAP_SWIZZLE_64B) &&
+         make_map_3d(&tsc, a.kv_scale, kBS, 1, a.num_blocks, kBS * 4, kBS * 4, kBS, 1, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
   } else {
     ok = ok &&
          make_map_3d(&tkv, a.cache, kR + kDR, kBS, a.num_blocks, (kR + kDR) * 2, (uint64_t)kBS * (kR + kDR) * 2, 64,
@@ -778,6 +779,7 @@ cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
                      kBS, CU_TENSOR_MAP_SWIZZLE_64B);
   }
   if (!ok) return cudaErrorInvalidValue;
+  if (!fp8) tsc = tkr;   // unused by the bf16 kernel
   static std::once_flag attr_once[2][64];
   int dev = 0;
   cudaGetDevice(&dev);
@@ -792,9 +794,9 @@ cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
   const uint64_t timeout_ns = 2000000000ull;
   const dim3 grid(2 * a.W * n_rg);
   if (fp8)
-    tc_decode_kernel<true><<<grid, threads_for<true>(), kSmemBytes, s>>>(tqr, tkv, tkr, a, n_rg, timeout_ns);
+    tc_decode_kernel<true><<<grid, threads_for<true>(), kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a, n_rg, timeout_ns);
   else
-    tc_decode_kernel<false><<<grid, threads_for<false>(), kSmemBytes, s>>>(tqr, tkv, tkr, a, n_rg, timeout_ns);
+    tc_decode_kernel<false><<<grid, threads_for<false>(), kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a, n_rg, timeout_ns);
   return cudaGetLastError();
 }
 
