@@ -5,44 +5,47 @@
 //  * The 128 query rows of a row group (Sq * H rows of one sequence, zero-padded) are
 //    the M = 128 rows of every MMA. Their fp32 output O[128 x 512] would fill all 512
 //    TMEM columns, so the two CTAs of the pair split the latent channels: CTA j owns
-//    latent channels [256 j, 256 j + 256) and RoPE channels [32 j, 32 j + 32).
-//  * TMEM per CTA (128 lanes = query rows): O [0, 256), scores S [256, 320),
+//    latent channels [256 j, 256 j + 256) and RoPE channels [32 j, 32 j + 32) of every
+//    MMA, for all 128 rows.
+//  * TMEM per CTA (128 lanes = query rows): O [0, 256), partial scores S [256, 320),
 //    probabilities P (bf16 pairs, double buffered) [320, 384), and the CTA's half of
 //    the absorbed query, latent part, as a TMEM A operand [384, 512).
 //  * Each CTA TMA-loads only its channel slice of every 64-token cache block
 //    (4 x [64 tok][64 ch] 128B-swizzled + [64 tok][32 ch] 64B-swizzled = 36 KB per
 //    stage, 4 stages). The query's RoPE part stays in shared memory (8 KB).
 //  * QK: S_j[128 x 64] = Q_j . C_j^T over the CTA's 288 channels (16 MMAs with A in
-//    TMEM + 2 with A in shared memory, K = 16 each).
-//  * Score exchange: the 8 softmax warps each own 32 rows x 32 columns of S. A warp
-//    stages its fp32 partial scores (4 KB) in shared memory and ships them with one
-//    bulk copy into the peer CTA, completing bytes on the peer's mbarrier; the peer's
-//    matching warp adds the two partials in the same order, so both CTAs hold the same
-//    full score. Two 32 KB buffers alternate roles: the one that received tile t - 1
-//    stages the outgoing partials of tile t + 1... precisely, buffer t & 1 receives
-//    tile t and buffer (t + 1) & 1 stages tile t; per-warp mbarriers tell the sender
-//    when the peer's buffer is free again.
-//  * Software pipeline of the softmax warps, iteration g: load S(g) and ship it;
-//    finish tile g - 1 (exponentials, P into TMEM); then combine tile g's partials and
-//    take its row maximum. The exchange of tile g overlaps the exponentials of g - 1.
-//    Two threads per query row (32 columns each) exchange their maxima through shared
-//    memory; the running maximum only moves when a tile raises it by more than 2^8,
-//    so O is rescaled rarely.
+//    TMEM + 2 with A in shared memory, K = 16 each). The full score is S_0 + S_1.
+//  * Row split of the softmax: CTA j normalises the 64 rows in TMEM lane quarters
+//    2 j and 2 j + 1 ("own" rows); the other 64 are the peer's. Per tile:
+//      - the 4 warps on the peer's quarters read those rows of S_j and store them with
+//        st.async straight into the peer's receive buffer (16 KB; bytes complete on
+//        the peer's mbarrier);
+//      - the 4 warps on the own quarters add the peer's partials to their own, take
+//        the row maximum (two warps per row, 32 columns each), the exponentials and
+//        the row sums, write P into TMEM and st.async the same bf16 rows (8 KB) plus
+//        one rescale factor per row to the peer;
+//      - the peer-quarter warps then write the received P rows into their TMEM and,
+//        when the owner moved a row's running maximum, rescale those O rows.
+//    Only 24.25 KB cross the pair per tile and direction, every exponential is taken
+//    once, and the exchange of a tile overlaps the exponentials of the previous one.
+//    The running maximum only moves when a tile raises it by more than 2^8, so O is
+//    rescaled rarely.
 //  * PV: O_j[128 x 256] += P[128 x 64] . C_j[64 x 256] with A = P from TMEM and B =
 //    the SAME shared-memory tile the QK used, read N-major (4 MMAs, N = 256). The MMA
 //    issuer runs QK(k) then PV(k - 2).
 //  * FP8 cache, exact: c_t = code_t * s_t with a per-token fp32 scale s_t. The
 //    producer TMA-loads the CTA's 256 e4m3 codes per token (16 KB) into the upper half
-//    of the stage and the bf16 RoPE key into its slot; two converter warps (one token row
-//    per thread) write the codes back as bf16 in place (every e4m3 value is exact in
-//    bf16) in the 128B-swizzled layout the bf16 path loads, and replace the RoPE key by
-//    kR_t / s_t split into bf16 hi + lo parts (2^-16 relative). The score MMAs then give
-//    S_t / s_t; the softmax multiplies each column by s_t, and P by s_t before PV
-//    (sum_t p_t s_t code_t = sum_t p_t c_t), with the row sum over the unscaled p_t.
-//  * Warp roles: warps 0-7 softmax / epilogue, warp 8 TMA producer, warp 9 TMEM
-//    allocator and single-thread MMA issuer, warps 10-11 FP8 converters; mbarrier
-//    pipelines between them. Every wait is bounded (timeout -> MLA_ERR_TIMEOUT,
-//    clean exit).
+//    of the stage, the bf16 RoPE key into its slot and the block's 64 scales; two
+//    converter warps (one token row per thread) write the codes back as bf16 in place
+//    (every e4m3 value is exact in bf16) in the 128B-swizzled layout the bf16 path
+//    loads, and replace the RoPE key by kR_t / s_t split into bf16 hi + lo parts
+//    (2^-16 relative). The score MMAs then give S_t / s_t; the softmax multiplies each
+//    column by s_t, and P by s_t before PV (sum_t p_t s_t code_t = sum_t p_t c_t), with
+//    the row sum over the unscaled p_t.
+//  * Warp roles: warps 0-7 softmax / exchange / epilogue, warp 8 TMA producer, warp 9
+//    TMEM allocator and single-thread MMA issuer, warps 10-11 FP8 converters; mbarrier
+//    pipelines between them. Every wait is bounded (timeout -> MLA_ERR_TIMEOUT, clean
+//    exit).
 // The work split over workers (CTA pairs) is the flat block list plan of mla_device.cuh.
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -61,35 +64,47 @@ using namespace ptx;
 
 constexpr int kR = 512, kDR = 64, kBS = 64;
 constexpr int kRows = 128;           // query rows per row group = MMA M
-constexpr int kMaxStages = 4;
+constexpr int kStages = 4;
 
 // shared memory layout, byte offsets from a 1024-aligned base
 constexpr uint32_t kKvLatChunk = kBS * 128;                      // [64 tok][64 ch] bf16, 128B swizzle
 constexpr uint32_t kKvRope = kBS * 64;                           // [64 tok][32 ch] bf16, 64B swizzle
+constexpr uint32_t kQRope = kRows * 64;                          // [128 rows][32 ch] bf16, 64B swizzle
+// Exchange buffers. Partial scores of 64 rows: 4 regions of [32 rows][32 cols] fp32;
+// probabilities of 64 rows: 4 regions of [32 rows][32 tokens] bf16 followed by 64 fp32
+// rescale factors. Each CTA stages what it sends in a buffer laid out like the peer's
+// receive buffer and moves every warp's region with one bulk copy.
+constexpr uint32_t kRxSRegion = 32 * 32 * 4;
+constexpr uint32_t kRxSBytes = 4 * kRxSRegion;                   // 16 KB
+constexpr uint32_t kRxPRegion = 32 * 32 * 2;
+constexpr uint32_t kRxPAlpha = 4 * kRxPRegion;                   // offset of the rescale factors
+constexpr uint32_t kRxPBytes = kRxPAlpha + 64 * 4;               // 8448
+constexpr uint32_t kLrxBytes = 64 * 4;                           // the peer's row sums of its rows
+constexpr uint32_t kCtlBytes = 4096;
 // bf16 stage: latent chunks + RoPE. FP8 stage: latent chunks + RoPE hi + RoPE lo + scales.
 template <bool kFp8> struct Geo {
-  static constexpr int kStages = kFp8 ? 3 : 4;
   static constexpr uint32_t kStageBytes = kFp8 ? 41984u : 36864u;
   static constexpr uint32_t kOffRopeLo = 4 * kKvLatChunk + kKvRope;   // FP8 only
   static constexpr uint32_t kOffScale = kOffRopeLo + kKvRope;         // FP8 only: 64 fp32
+  static constexpr uint32_t kOffKv = 0;
+  static constexpr uint32_t kOffQr = kStages * kStageBytes;
+  static constexpr uint32_t kRxSBufs = kFp8 ? 1 : 2;             // receive buffers for partial scores
+  static constexpr uint32_t kOffRxS = kOffQr + kQRope;
+  static constexpr uint32_t kOffRxP = kOffRxS + kRxSBufs * kRxSBytes;   // one receive buffer for P
+  static constexpr uint32_t kOffTxS = kOffRxP + kRxPBytes;             // staging of outgoing scores
+  static constexpr uint32_t kOffTxP = kOffTxS + kRxSBytes;             // ... and probabilities
+  static constexpr uint32_t kOffCtl = kOffTxP + kRxPBytes;
+  static constexpr uint32_t kSmemBytes = kOffCtl + kCtlBytes + 1024;   // + alignment slack
 };
 static_assert(Geo<true>::kOffScale + 256 <= Geo<true>::kStageBytes && Geo<true>::kStageBytes % 1024 == 0, "fp8 stage");
-constexpr uint32_t kQRope = kRows * 64;                          // [128 rows][32 ch] bf16, 64B swizzle
-constexpr uint32_t kXBytes = kRows * 64 * 4;                     // partial scores [128 rows][64] fp32
-constexpr uint32_t kXChunk = kXBytes / 8;                        // one softmax warp's 32 rows x 32 cols
-constexpr uint32_t kOffKv = 0;
-constexpr uint32_t kOffQr = 4 * 36864;   // after the stages (both cache types use <= 147456 bytes)
-static_assert(Geo<true>::kStages * Geo<true>::kStageBytes <= kOffQr, "stages fit");
-constexpr uint32_t kOffX = kOffQr + kQRope;                      // two exchange buffers
-constexpr uint32_t kOffCtl = kOffX + 2 * kXBytes;
-constexpr uint32_t kCtlBytes = 4096;
-constexpr uint32_t kSmemBytes = kOffCtl + kCtlBytes + 1024;      // + alignment slack
-static_assert(kOffQr % 1024 == 0 && kOffX % 1024 == 0, "buffers need 1024-byte alignment");
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(Geo<false>::kOffQr % 1024 == 0 && Geo<true>::kOffQr % 1024 == 0, "buffers need 1024-byte alignment");
+static_assert(Geo<false>::kSmemBytes <= 232448 && Geo<true>::kSmemBytes <= 232448, "shared memory budget");
+static_assert(kRxPBytes % 16 == 0 && Geo<true>::kOffTxS % 16 == 0 && Geo<false>::kOffTxS % 16 == 0,
+              "bulk copies need 16-byte alignment");
 
 // TMEM columns (32-bit lanes x columns; lane = query row)
 constexpr uint32_t kTmemO = 0;       // 256: this CTA's output channels
-constexpr uint32_t kTmemS = 256;     // 64: scores of the current tile
+constexpr uint32_t kTmemS = 256;     // 64: partial scores of the current tile
 constexpr uint32_t kTmemP = 320;     // 2 x 32: probabilities, bf16 pairs
 constexpr uint32_t kTmemQ = 384;     // 128: absorbed query, this CTA's 256 latent channels
 constexpr uint32_t kTmemCols = 512;
@@ -107,24 +122,28 @@ constexpr uint32_t kFp8StageTx = kFp8CodeBytes + kKvRope + kBS * 4;   // codes, 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only if the max grows > 2^8
 
 struct Ctl {
-  uint64_t kv_full[kMaxStages];
-  uint64_t kv_empty[kMaxStages];
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t kv_ready[kStages];   // FP8: the converted bf16 tile is in place
+  uint64_t cv_loaded[kStages];  // FP8: every converter thread holds its codes in registers
   uint64_t q_full, q_empty;
   uint64_t s_full, s_empty;
-  uint64_t p_full[2];
+  uint64_t p_full[2];       // P of tile t (both row halves) is in TMEM slot t & 1, O rescaled
   uint64_t pv_done[2];      // PV of tile t completes a phase of pv_done[t & 1]
-  uint64_t rx_full[2];      // exchange buffer b holds the peer's partials of the next tile t, t & 1 == b
-  uint64_t tx_ok[8][2];     // per warp: the peer's buffer b may take our next partials
-  uint64_t mx[4];           // the two warps sharing 32 rows published their tile maxima
-  uint64_t lx[4];           // ... their row sums
-  uint64_t kv_ready[kMaxStages];   // FP8: the converted bf16 tile is in place
-  uint64_t cv_loaded[kMaxStages];  // FP8: every converter thread holds its codes in registers
+  uint64_t rxs_full[2];     // the peer's partial scores of tile t landed in buffer t % kRxSBufs
+  uint64_t rxp_full;        // the peer's probabilities and rescale factors of the next tile landed
+  uint64_t txs_ok[2];       // the peer has read the partial scores we last sent into its buffer b
+  uint64_t txp_ok;          // ... the probabilities
+  uint64_t mx[2];           // the two warps sharing 32 own rows published their tile maxima
+  uint64_t lx[2];           // ... their row sums
+  uint64_t lrx_full[2];     // the peer's row sums of segment s, s & 1 == b, have landed
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
   WorkerPlan plan;
-  float mbuf[2][2][kRows];  // [tile parity][half][row]
-  float lbuf[2][kRows];     // [half][row]
+  float mbuf[2][2][64];     // [tile parity][half][own row]
+  float lbuf[2][64];        // [half][own row]
+  float lrx[2][64];         // [segment parity][peer's own row]: written by the peer
 };
 static_assert(sizeof(Ctl) <= kCtlBytes, "control block too large");
 
@@ -146,13 +165,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
     tc_decode_kernel(const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_sc,
                      const DecodeArgs a, const int n_rg, const uint64_t timeout_ns) {
-  constexpr int kStages = Geo<kFp8>::kStages;
-  constexpr uint32_t kStageBytes = Geo<kFp8>::kStageBytes;
+  using G = Geo<kFp8>;
+  constexpr uint32_t kStageBytes = G::kStageBytes;
+  constexpr uint32_t kOffKv = G::kOffKv;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  Ctl& ctl = *reinterpret_cast<Ctl*>(smem + kOffCtl);
+  Ctl& ctl = *reinterpret_cast<Ctl*>(smem + G::kOffCtl);
   const uint32_t sKv = smem_u32(smem + kOffKv);
-  const uint32_t sQr = smem_u32(smem + kOffQr);
+  const uint32_t sQr = smem_u32(smem + G::kOffQr);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
@@ -173,12 +193,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
     for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&ctl.p_full[i]), kSoftmaxThreads);
     for (int i = 0; i < 2; ++i) mbar_init(smem_u32(&ctl.pv_done[i]), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&ctl.rx_full[i]), 1);
-      mbar_arrive_expect_tx(smem_u32(&ctl.rx_full[i]), kXBytes);   // armed for tiles 0 and 1
-    }
-    for (int i = 0; i < 8; ++i)
-      for (int j = 0; j < 2; ++j) mbar_init(smem_u32(&ctl.tx_ok[i][j]), 1);
-    for (int i = 0; i < 4; ++i) {
+      // receive barriers: one local arrival plus the peer's bytes; armed for tiles (segments) 0 and 1
+      mbar_init(smem_u32(&ctl.rxs_full[i]), 1);
+      mbar_arrive_expect_tx(smem_u32(&ctl.rxs_full[i]), kRxSBytes);
+      mbar_init(smem_u32(&ctl.lrx_full[i]), 1);
+      mbar_arrive_expect_tx(smem_u32(&ctl.lrx_full[i]), kLrxBytes);
+      mbar_init(smem_u32(&ctl.txs_ok[i]), 4);   // one arrival per consuming warp of the peer
       mbar_init(smem_u32(&ctl.mx[i]), 64);
       mbar_init(smem_u32(&ctl.lx[i]), 64);
     }
@@ -186,6 +206,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
       mbar_init(smem_u32(&ctl.kv_ready[i]), kConvThreads);
       mbar_init(smem_u32(&ctl.cv_loaded[i]), kConvThreads);
     }
+    mbar_init(smem_u32(&ctl.rxp_full), 1);
+    mbar_arrive_expect_tx(smem_u32(&ctl.rxp_full), kRxPBytes);   // armed for tile 0
+    mbar_init(smem_u32(&ctl.txp_ok), 4);
     mbar_init(smem_u32(&ctl.drain), 1);
     ctl.abort = 0;
     fence_mbarrier_init_cluster();
@@ -403,20 +426,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
       if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
     }
   } else {
-    // ------------------------------------------------------------------ softmax + epilogue
-    const int st_idx = threadIdx.x;                    // 0..255
-    const int row = st_idx & (kRows - 1);              // TMEM lane / query row in the group
-    const int half = st_idx >> 7;                      // columns [32 half, 32 half + 32)
-    const int quad = warp & 3;                         // the TMEM lane quarter of this warp
+    // ------------------------------------------------------------------ softmax, exchange, epilogue
+    const int quad = warp & 3;                          // the TMEM lane quarter of this warp
+    const int half = warp >> 2;                         // score columns [32 half, +32), O columns [128 half, +128)
+    const bool own = (quad >> 1) == (int)rank;          // this CTA normalises the rows of this quarter
+    const int row = quad * 32 + lane;                   // TMEM lane = query row in the group
+    const int orow = (quad & 1) * 32 + lane;            // the row among the 64 that one CTA normalises
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    // exchange: this warp's 4 KB chunk of an exchange buffer; 16-byte pieces of a lane's
-    // 128-byte row XOR-swizzled by the lane to spread shared-memory banks
-    const uint32_t chunk_off = kOffX + warp * kXChunk + lane * 128;
-    const uint32_t peer_x0 = mapa(smem_u32(smem + kOffX + warp * kXChunk), peer);
-    const uint32_t peer_rx_full0 = mapa(smem_u32(&ctl.rx_full[0]), peer);
-    const uint32_t peer_rx_full1 = mapa(smem_u32(&ctl.rx_full[1]), peer);
-    const uint32_t peer_tx_ok0 = mapa(smem_u32(&ctl.tx_ok[warp][0]), peer);
-    const uint32_t peer_tx_ok1 = mapa(smem_u32(&ctl.tx_ok[warp][1]), peer);
+    // Exchange partners: own warp w of one CTA and peer warp w of the other (same quarter,
+    // same column half) share region (quad & 1) * 2 + half of each receive buffer.
+    const int region = (quad & 1) * 2 + half;
+    const bool leader = lane == 0 && half == 0 && (quad & 1) == 0;   // one thread per group re-arms
+    constexpr uint32_t kNbS = G::kRxSBufs;
+    // this warp's region: row `lane` of it in the receive and the staging buffers
+    const uint32_t rxs_me = smem_u32(smem + G::kOffRxS) + region * kRxSRegion + lane * 128;
+    const uint32_t txs_me = smem_u32(smem + G::kOffTxS) + region * kRxSRegion + lane * 128;
+    const uint32_t rxp_me = smem_u32(smem + G::kOffRxP) + region * kRxPRegion + lane * 64;
+    const uint32_t txp_me = smem_u32(smem + G::kOffTxP) + region * kRxPRegion + lane * 64;
+    const uint32_t alpha_off = kRxPAlpha + (quad & 1) * 128;   // this quarter's 32 rescale factors
+    const uint32_t alpha_me = smem_u32(smem + G::kOffRxP) + alpha_off + lane * 4;
+    // 16-byte pieces of a lane's row are XOR-swizzled so that 8 consecutive lanes hit
+    // distinct banks: partial scores 128 B per row, probabilities 64 B per row
+    auto s_piece = [&](int c) { return (uint32_t)((c ^ (lane & 7)) << 4); };
+    auto p_piece = [&](int c) { return (uint32_t)((c ^ ((lane >> 1) & 3)) << 4); };
     const int grow = rg * kRows + row;
     const bool valid_row = grow < a.rows;
     const int s_idx = valid_row ? grow / a.H : 0;
@@ -432,11 +464,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
     auto wait_peer = [&](uint32_t bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait<true>(bar, parity, abort, timeout_ns));
     };
+    // lane 0 waits for a barrier the peer arrives on (a buffer handed back); the warp follows
+    auto wait_remote_arrival = [&](uint32_t bar, uint32_t parity) {
+      bool r = true;
+      if (lane == 0) r = mbar_wait<false>(bar, parity, abort, timeout_ns);
+      return __all_sync(0xffffffffu, r);
+    };
     // PV(j) done. Valid while PV(j - 2) is complete and PV(j + 2) cannot be (its P is
-    // not written yet): callers only wait for PVs of the current segment.
+    // not written yet): callers only wait for PVs of the current segment, in order.
     auto wait_pv = [&](uint32_t j) { return wait_local(smem_u32(&ctl.pv_done[j & 1]), (j >> 1) & 1); };
+    // O rows of this warp's lanes, its 128 columns, times alpha (all earlier PVs complete)
+    auto rescale_o = [&](float alpha) {
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t v[16];
+        const uint32_t ta = tmem + lane_off + kTmemO + 128 * half + 16 * c;
+        tmem_ld16(ta, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+        tmem_st16(ta, v);
+      }
+      tmem_wait_st();
+    };
+    // this warp's 32 partial-score columns of the current tile, out of TMEM
+    auto load_s = [&](uint32_t gt, uint32_t* sv) {
+      if (!wait_local(smem_u32(&ctl.s_full), gt & 1)) return false;
+      tc_fence_after();
+      tmem_ld16(tmem + lane_off + kTmemS + 32 * half, sv);
+      tmem_ld16(tmem + lane_off + kTmemS + 32 * half + 16, sv + 16);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&ctl.s_empty));
+      return true;
+    };
     while (ok && it.next(sg)) {
-      // this segment's absorbed query, latent half of this CTA, into TMEM
+      // this segment's absorbed query, latent half of this CTA, into TMEM (all 128 rows)
       ok = wait_local(smem_u32(&ctl.q_empty), (seg & 1) ^ 1);
       if (!ok) break;
       {
@@ -458,71 +521,83 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
         tc_fence_before();
         mbar_arrive(smem_u32(&ctl.q_full));
       }
-      int n_row = valid_row ? (a.causal ? sg.Lc - a.Sq + 1 + s_idx : sg.Lc) : 0;
-      if (n_row < 0) n_row = 0;
-      float m_run = -INFINITY, l_run = 0.f;
       const int n = sg.tile_end - sg.tile_begin;
       const int last_tile = (sg.Lc + kBS - 1) / kBS - 1;
-      float x[32];          // scaled scores (log2 units) of the tile awaiting its exponentials
-      float mt = -INFINITY; // that tile's row maximum
-      for (int li = 0; li <= n; ++li) {
-        const uint32_t gt = g + li;   // tile of stage A / B1 (g + li), B2 handles gt - 1
-        uint32_t sv[32];
-        if (li < n) {
-          // ---- A: scores of tile gt out of TMEM, staged and shipped to the peer
-          ok = wait_local(smem_u32(&ctl.s_full), gt & 1);
+      float m_run = -INFINITY, l_run = 0.f;   // own rows: running maximum (log2 units) and sum
+      if (own) {
+        int n_row = valid_row ? (a.causal ? sg.Lc - a.Sq + 1 + s_idx : sg.Lc) : 0;
+        if (n_row < 0) n_row = 0;
+        for (int li = 0; li < n; ++li) {
+          const uint32_t gt = g + li, b = gt & 1;
+          const int tile = sg.tile_begin + li;
+          uint32_t sv[32];
+          ok = load_s(gt, sv);
           if (!ok) break;
-          tc_fence_after();
-          tmem_ld16(tmem + lane_off + kTmemS + 32 * half, sv);
-          tmem_ld16(tmem + lane_off + kTmemS + 32 * half + 16, sv + 16);
-          tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(smem_u32(&ctl.s_empty));
-          // the peer's buffer gt & 1 is free once its copy of tile gt - 1 left it
-          if (lane == 0) {
-            const uint32_t par = ((((gt + 1) >> 1) - 1u) & 1u);
-            ok = mbar_wait<true>(smem_u32(&ctl.tx_ok[warp][gt & 1]), par, abort, timeout_ns);
+          // ---- the peer's partials of our rows; full scores; row maximum
+          const uint32_t bs = gt % kNbS;
+          ok = wait_peer(smem_u32(&ctl.rxs_full[bs]), (gt / kNbS) & 1);
+          if (!ok) break;
+          const uint32_t rx = rxs_me + bs * kRxSBytes;
+          float x[32];
+          float mh = -INFINITY;
+          const int valid = min(max(n_row - tile * kBS - 32 * half, 0), 32);   // of my 32 columns
+          const float4* cs = nullptr;   // FP8: token scales of my columns
+          if constexpr (kFp8) {
+            const uint32_t stg = gt % kStages;
+            int dummy = 0;
+            mbar_wait<false>(smem_u32(&ctl.kv_ready[stg]), (gt / kStages) & 1, &dummy, timeout_ns);
+            cs = reinterpret_cast<const float4*>(smem + kOffKv + stg * kStageBytes + G::kOffScale + 128 * half);
           }
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          const uint32_t stage_off = chunk_off + ((gt + 1) & 1) * kXBytes;   // outgoing: buffer (gt + 1) & 1
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(smem + stage_off + ((c ^ (lane & 7)) << 4)) =
-                make_uint4(sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            bulk_copy_to_peer(peer_x0 + (gt & 1) * kXBytes, smem_u32(smem + kOffX + ((gt + 1) & 1) * kXBytes +
-                                                                        warp * kXChunk),
-                              kXChunk, (gt & 1) ? peer_rx_full1 : peer_rx_full0);
-            bulk_commit_group();
+          for (int c = 0; c < 8; ++c) {
+            uint4 v;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(rx + s_piece(c)));
+            const float r4[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                                 __uint_as_float(v.w)};
+            float c4[4] = {1.f, 1.f, 1.f, 1.f};
+            if constexpr (kFp8) {
+              const float4 t = cs[c];
+              c4[0] = t.x;
+              c4[1] = t.y;
+              c4[2] = t.z;
+              c4[3] = t.w;
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int k = 4 * c + i;
+              const float sc = (__uint_as_float(sv[k]) + r4[i]) * c4[i] * scale_log2;
+              x[k] = k < valid ? sc : -INFINITY;
+              mh = fmaxf(mh, x[k]);
+            }
           }
-        }
-        if (li > 0) {
-          // ---- B2: exponentials of tile gt - 1, P into TMEM
-          const uint32_t gp = gt - 1;
-          const int tile = sg.tile_begin + li - 1;
+          ctl.mbuf[b][half][orow] = mh;   // depends on every value read from the receive buffer
+          __syncwarp();
+          // the peer may refill our region of buffer bs (tile gt + kNbS)
+          if (lane == 0) mbar_arrive_remote_cta(mapa(smem_u32(&ctl.txs_ok[bs]), peer));
+          if (leader) mbar_arrive_expect_tx(smem_u32(&ctl.rxs_full[bs]), kRxSBytes);
+          mbar_arrive(smem_u32(&ctl.mx[quad & 1]));
+          ok = wait_local(smem_u32(&ctl.mx[quad & 1]), gt & 1);
+          if (!ok) break;
+          const float mt = fmaxf(ctl.mbuf[b][0][orow], ctl.mbuf[b][1][orow]);
+          // ---- exponentials, P into TMEM and to the peer
           const bool grow_max = mt > m_run + kRescaleThreshold;
           const bool rescale = grow_max && m_run != -INFINITY;
           const float alpha = rescale ? ex2_approx(m_run - mt) : 1.f;
-          if (__any_sync(0xffffffffu, rescale)) {
-            // O holds this segment's tiles before gp: wait for their last two PVs (older
-            // ones are known complete), then scale in place
-            ok = (gp < g + 2 || wait_pv(gp - 2)) && wait_pv(gp - 1);
+          // P slot b is free once PV(gt - 2) has completed
+          if (li >= 2) {
+            ok = wait_pv(gt - 2);
             if (!ok) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
-              uint32_t v[16];
-              const uint32_t ta = tmem + lane_off + kTmemO + 128 * half + 16 * c;
-              tmem_ld16(ta, v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-              tmem_st16(ta, v);
+          }
+          if (__any_sync(0xffffffffu, rescale)) {
+            // O holds this segment's tiles before gt: wait for the last PV, then scale
+            if (li >= 1) {
+              ok = wait_pv(gt - 1);
+              if (!ok) break;
             }
-            tmem_wait_st();
+            tc_fence_after();
+            rescale_o(alpha);
           }
           if (grow_max) {
             l_run *= alpha;
@@ -533,16 +608,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
           const bool any = m_run != -INFINITY;
           float pcs[32];     // FP8: P columns carry the token scale into PV (0 for unseen tokens)
           if constexpr (kFp8) {
-            const int valid_p = min(max(n_row - tile * kBS - 32 * half, 0), 32);
-            const float4* cs = reinterpret_cast<const float4*>(smem + kOffKv + (gp % kStages) * kStageBytes +
-                                                               Geo<kFp8>::kOffScale + 128 * half);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               const float4 v = cs[c];
-              pcs[4 * c] = 4 * c < valid_p ? v.x : 0.f;
-              pcs[4 * c + 1] = 4 * c + 1 < valid_p ? v.y : 0.f;
-              pcs[4 * c + 2] = 4 * c + 2 < valid_p ? v.z : 0.f;
-              pcs[4 * c + 3] = 4 * c + 3 < valid_p ? v.w : 0.f;
+              pcs[4 * c] = 4 * c < valid ? v.x : 0.f;
+              pcs[4 * c + 1] = 4 * c + 1 < valid ? v.y : 0.f;
+              pcs[4 * c + 2] = 4 * c + 2 < valid ? v.z : 0.f;
+              pcs[4 * c + 3] = 4 * c + 3 < valid ? v.w : 0.f;
             }
           }
 #pragma unroll
@@ -556,97 +628,171 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
               pk[k >> 1] = pack_bf16x2(p0, p1);
           }
           l_run += psum;
-          tmem_st16(tmem + lane_off + kTmemP + 32 * (gp & 1) + 16 * half, pk);
-          tmem_wait_st();
+          tmem_st16(tmem + lane_off + kTmemP + 32 * b + 16 * half, pk);
+          // stage the P row (and the rescale factor) like the peer's receive buffer; our
+          // previous copy out of the staging region must have finished reading it
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(txp_me + p_piece(c)), "r"(pk[4 * c]),
+                         "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                         : "memory");
+          if (half == 0)
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(smem_u32(smem + G::kOffTxP) + alpha_off + lane * 4),
+                         "f"(alpha)
+                         : "memory");
+          fence_proxy_async_smem();
+          // the peer's receive buffer is free once it has read tile gt - 1
+          if (gt >= 1) {
+            ok = wait_remote_arrival(smem_u32(&ctl.txp_ok), (gt - 1) & 1);
+            if (!ok) break;
+          }
+          if (lane == 0) {
+            const uint32_t bar = mapa(smem_u32(&ctl.rxp_full), peer);
+            const uint32_t rbase = region * kRxPRegion;
+            bulk_copy_to_peer(mapa(smem_u32(smem + G::kOffRxP) + rbase, peer), smem_u32(smem + G::kOffTxP) + rbase,
+                              kRxPRegion, bar);
+            if (half == 0)
+              bulk_copy_to_peer(mapa(smem_u32(smem + G::kOffRxP) + alpha_off, peer),
+                                smem_u32(smem + G::kOffTxP) + alpha_off, 128, bar);
+            bulk_commit_group();
+          }
           // Slots past the sequence end in its last block may hold anything (NaN): zero
           // those token rows of this CTA's latent slice before the PV reads them.
           const int tail = sg.Lc % kBS;
           if (tile == last_tile && tail != 0) {
-            const uint32_t stg = gp % kStages;
+            const uint32_t stg = gt % kStages;
             int dummy = 0;
-            mbar_wait<false>(smem_u32(kFp8 ? &ctl.kv_ready[stg] : &ctl.kv_full[stg]), (gp / kStages) & 1, &dummy,
+            mbar_wait<false>(smem_u32(kFp8 ? &ctl.kv_ready[stg] : &ctl.kv_full[stg]), (gt / kStages) & 1, &dummy,
                              timeout_ns);
             uint8_t* base = smem + kOffKv + stg * kStageBytes;
             const int per_chunk = (kBS - tail) * 8;          // 16-byte pieces per chunk
-            for (int i = st_idx; i < 4 * per_chunk; i += kSoftmaxThreads) {
+            const int t0 = (quad & 1) * 32 + half * 64 + lane;   // 0..127 over the own warps
+            for (int i = t0; i < 4 * per_chunk; i += 128) {
               const int chunk = i / per_chunk, rem = i % per_chunk;
               *reinterpret_cast<uint4*>(base + chunk * kKvLatChunk + (tail + rem / 8) * 128 + (rem % 8) * 16) =
                   make_uint4(0u, 0u, 0u, 0u);
             }
             fence_proxy_async_smem();
           }
+          tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(smem_u32(&ctl.p_full[gp & 1]));
+          mbar_arrive(smem_u32(&ctl.p_full[b]));
         }
-        if (li < n) {
-          // ---- B1: the peer's partials of tile gt; full scores; row maximum
-          const int tile = sg.tile_begin + li;
+      } else {
+        // Peer quarters: two in-order streams served as they become ready -- ship the
+        // partial scores of each tile to the peer, and take the peer's P rows of each tile
+        // into TMEM. Lane 0 polls, the warp follows its choice.
+        int ship = 0, recv = 0;   // next segment-local tile of each stream
+        uint32_t spins = 0;
+        uint64_t t_idle = 0;
+        while (recv < n) {
+          int act = 0;
           if (lane == 0) {
-            // our outgoing copy no longer reads buffer (gt + 1) & 1: the peer may fill it
-            bulk_wait_group_read<0>();
-            mbar_arrive_remote(((gt + 1) & 1) ? peer_tx_ok1 : peer_tx_ok0);
-          }
-          ok = wait_peer(smem_u32(&ctl.rx_full[gt & 1]), (gt >> 1) & 1);
-          if (!ok) break;
-          if (st_idx == 0) mbar_arrive_expect_tx(smem_u32(&ctl.rx_full[gt & 1]), kXBytes);   // tile gt + 2
-          const uint32_t in_off = chunk_off + (gt & 1) * kXBytes;
-          const int valid = min(max(n_row - tile * kBS - 32 * half, 0), 32);   // of my 32 columns
-          float colsc[32];   // FP8: token scales of my columns (1 for the bf16 cache)
-          if constexpr (kFp8) {
-            const uint32_t stg = gt % kStages;
-            int dummy = 0;
-            mbar_wait<false>(smem_u32(&ctl.kv_ready[stg]), (gt / kStages) & 1, &dummy, timeout_ns);
-            const float4* cs = reinterpret_cast<const float4*>(smem + kOffKv + stg * kStageBytes +
-                                                               Geo<kFp8>::kOffScale + 128 * half);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const float4 v = cs[c];
-              colsc[4 * c] = v.x;
-              colsc[4 * c + 1] = v.y;
-              colsc[4 * c + 2] = v.z;
-              colsc[4 * c + 3] = v.w;
+            if (ship < n && mbar_test_wait(smem_u32(&ctl.s_full), (g + ship) & 1))
+              act = 1;
+            else if (recv < ship && mbar_test_wait_cluster(smem_u32(&ctl.rxp_full), (g + recv) & 1))
+              act = 2;
+            else if ((++spins & 255u) == 0u) {
+              const uint64_t now = globaltimer();
+              if (*abort) act = 3;
+              else if (t_idle == 0) t_idle = now;
+              else if (now - t_idle > timeout_ns) { *abort = 1; act = 3; }
             }
-          } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k) colsc[k] = 1.f;
+            if (act == 1 || act == 2) { spins = 0; t_idle = 0; }
           }
-          float mh = -INFINITY;
+          act = __shfl_sync(0xffffffffu, act, 0);
+          if (act == 3) { ok = false; break; }
+          if (act == 1) {
+            const uint32_t gt = g + ship, bs = gt % kNbS;
+            uint32_t sv[32];
+            ok = load_s(gt, sv);
+            if (!ok) break;
+            // stage the rows; our previous copy out of the staging region must be done reading
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4*>(smem + in_off + ((c ^ (lane & 7)) << 4));
-            const float r4[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
-                                 __uint_as_float(v.w)};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int k = 4 * c + i;
-              const float sc = (__uint_as_float(sv[k]) + r4[i]) * colsc[k] * scale_log2;
-              x[k] = k < valid ? sc : -INFINITY;
-              mh = fmaxf(mh, x[k]);
+            for (int c = 0; c < 8; ++c)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(txs_me + s_piece(c)), "r"(sv[4 * c]),
+                           "r"(sv[4 * c + 1]), "r"(sv[4 * c + 2]), "r"(sv[4 * c + 3])
+                           : "memory");
+            fence_proxy_async_smem();
+            // the peer's receive buffer bs is free once it has read tile gt - kNbS
+            if (gt >= kNbS) {
+              ok = wait_remote_arrival(smem_u32(&ctl.txs_ok[bs]), ((gt / kNbS) + 1) & 1);
+              if (!ok) break;
             }
+            if (lane == 0) {
+              const uint32_t rbase = region * kRxSRegion;
+              bulk_copy_to_peer(mapa(smem_u32(smem + G::kOffRxS) + bs * kRxSBytes + rbase, peer),
+                                smem_u32(smem + G::kOffTxS) + rbase, kRxSRegion,
+                                mapa(smem_u32(&ctl.rxs_full[bs]), peer));
+              bulk_commit_group();
+            }
+            ++ship;
+          } else if (act == 2) {
+            const uint32_t gp = g + recv, b = gp & 1;
+            ok = wait_peer(smem_u32(&ctl.rxp_full), gp & 1);   // completes at once
+            if (!ok) break;
+            uint32_t pk[16];
+            const uint32_t rx = rxp_me;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(pk[4 * c]), "=r"(pk[4 * c + 1]), "=r"(pk[4 * c + 2]), "=r"(pk[4 * c + 3])
+                           : "r"(rx + p_piece(c)));
+            float alpha;
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(alpha) : "r"(alpha_me));
+            if (recv >= 2) {   // P slot b held tile gp - 2 of this segment
+              ok = wait_pv(gp - 2);
+              if (!ok) break;
+            }
+            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+              if (recv >= 1) {
+                ok = wait_pv(gp - 1);
+                if (!ok) break;
+              }
+              tc_fence_after();
+              rescale_o(alpha);
+            }
+            tmem_st16(tmem + lane_off + kTmemP + 32 * b + 16 * half, pk);   // consumes the loaded rows
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote_cta(mapa(smem_u32(&ctl.txp_ok), peer));
+            if (leader) mbar_arrive_expect_tx(smem_u32(&ctl.rxp_full), kRxPBytes);   // tile gp + 1
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(smem_u32(&ctl.p_full[b]));
+            ++recv;
           }
-          ctl.mbuf[gt & 1][half][row] = mh;
-          mbar_arrive(smem_u32(&ctl.mx[quad]));
-          ok = wait_local(smem_u32(&ctl.mx[quad]), gt & 1);
-          if (!ok) break;
-          mt = fmaxf(ctl.mbuf[gt & 1][0][row], ctl.mbuf[gt & 1][1][row]);
         }
       }
       if (!ok) break;
       g += n;
 
       // epilogue: O / l -> out (single split) or the normalised partial (several splits).
-      // Known complete: the PV three tiles before the last; wait for the last three PVs
-      // of this segment in order.
-      for (uint32_t j = (n >= 3 ? g - 3 : g - n); ok && j < g; ++j) ok = wait_pv(j);
+      // PVs up to g - 3 were waited for above; wait for the last two in order.
+      for (uint32_t j = (n >= 2 ? g - 2 : g - 1); ok && j < g; ++j) ok = wait_pv(j);
       if (!ok) break;
       tc_fence_after();
-      ctl.lbuf[half][row] = l_run;
-      mbar_arrive(smem_u32(&ctl.lx[quad]));
-      ok = wait_local(smem_u32(&ctl.lx[quad]), seg & 1);
-      if (!ok) break;
-      const float l_tot = ctl.lbuf[0][row] + ctl.lbuf[1][row];
+      float l_tot;
+      if (own) {
+        ctl.lbuf[half][orow] = l_run;
+        mbar_arrive(smem_u32(&ctl.lx[quad & 1]));
+        ok = wait_local(smem_u32(&ctl.lx[quad & 1]), seg & 1);
+        if (!ok) break;
+        l_tot = ctl.lbuf[0][orow] + ctl.lbuf[1][orow];
+        if (half == 0)
+          st_async_b32(mapa(smem_u32(&ctl.lrx[seg & 1][orow]), peer), __float_as_uint(l_tot),
+                       mapa(smem_u32(&ctl.lrx_full[seg & 1]), peer));
+      } else {
+        ok = wait_peer(smem_u32(&ctl.lrx_full[seg & 1]), (seg >> 1) & 1);
+        if (!ok) break;
+        l_tot = ctl.lrx[seg & 1][orow];
+        __syncwarp();
+        if (leader) mbar_arrive_expect_tx(smem_u32(&ctl.lrx_full[seg & 1]), kLrxBytes);   // segment seg + 2
+      }
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-      const float lse_v = l_tot > 0.f ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
       const size_t qrow = (size_t)sg.b * a.rows + grow;
       const bool direct = sg.splits == 1;
       const size_t prow = (size_t)(w + sg.b) * a.rows + grow;
@@ -679,20 +825,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
                             __uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
         }
       }
-      if (valid_row && rank == 0 && half == 0) {
+      if (own && half == 0 && valid_row) {
+        const float lse_v = l_tot > 0.f ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
         if (direct)
           a.lse[qrow] = lse_v;
         else
           a.lse_part[prow] = lse_v;
       }
-      if (sg.split == 0 && rg == 0 && rank == 0 && st_idx == 0) {
+      if (sg.split == 0 && rg == 0 && rank == 0 && threadIdx.x == 0) {
         a.meta[2 * sg.b] = sg.first_worker;
         a.meta[2 * sg.b + 1] = sg.splits;
       }
       tc_fence_before();
       ++seg;
     }
-    if (lane == 0) bulk_wait_group_read<0>();
+    if (lane == 0) bulk_wait_group_read<0>();   // staging regions stay valid until read
     if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
   }
 
@@ -786,17 +933,19 @@ cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
   cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once[fp8 ? 1 : 0][dev & 63], [&] {
     attr_err = fp8 ? cudaFuncSetAttribute(tc_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          kSmemBytes)
+                                          Geo<true>::kSmemBytes)
                    : cudaFuncSetAttribute(tc_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          kSmemBytes);
+                                          Geo<false>::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
   const uint64_t timeout_ns = 2000000000ull;
   const dim3 grid(2 * a.W * n_rg);
   if (fp8)
-    tc_decode_kernel<true><<<grid, threads_for<true>(), kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a, n_rg, timeout_ns);
+    tc_decode_kernel<true><<<grid, threads_for<true>(), Geo<true>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a, n_rg,
+                                                                                    timeout_ns);
   else
-    tc_decode_kernel<false><<<grid, threads_for<false>(), kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a, n_rg, timeout_ns);
+    tc_decode_kernel<false><<<grid, threads_for<false>(), Geo<false>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a, n_rg,
+                                                                                       timeout_ns);
   return cudaGetLastError();
 }
 
