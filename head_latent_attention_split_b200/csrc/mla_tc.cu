@@ -427,28 +427,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
     }
   } else {
     // ------------------------------------------------------------------ softmax, exchange, epilogue
-    const int quad = warp & 3;                          // the TMEM lane quarter of this warp
-    const int half = warp >> 2;                         // score columns [32 half, +32), O columns [128 half, +128)
-    const bool own = (quad >> 1) == (int)rank;          // this CTA normalises the rows of this quarter
-    const int row = quad * 32 + lane;                   // TMEM lane = query row in the group
-    const int orow = (quad & 1) * 32 + lane;            // the row among the 64 that one CTA normalises
-    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    // Exchange partners: own warp w of one CTA and peer warp w of the other (same quarter,
-    // same column half) share region (quad & 1) * 2 + half of each receive buffer.
-    const int region = (quad & 1) * 2 + half;
-    const bool leader = lane == 0 && half == 0 && (quad & 1) == 0;   // one thread per group re-arms
+    // Row split: in every TMEM lane quarter q, lanes [32 q + 16 rank, +16) hold this CTA's own
+    // rows and the other 16 lanes the peer's. Warp q (0-3) works on the own lanes of quarter
+    // q, warp q + 4 on the peer lanes, so both kinds of work spread over the four SM
+    // sub-partitions. With the 16-lane TMEM access shape, thread t and t + 16 share row
+    // t & 15 of the warp's lanes: columns [0, 32) and [32, 64) of a tile.
+    const int quad = warp & 3;
+    const bool own = warp < 4;
+    const int rr = lane & 15;                           // row within the warp's 16 lanes
+    const int hf = lane >> 4;                           // column half of the tile / of O
+    const int lbase = quad * 32 + 16 * (own ? (int)rank : (int)peer);
+    const uint32_t lane_off = (uint32_t)lbase << 16;
+    const int row = lbase + rr;                         // TMEM lane = query row in the group
+    const int orow = quad * 16 + rr;                    // the row among the 64 its owner normalises
+    const bool leader = lane == 0 && quad == 0;         // one thread per role re-arms
     constexpr uint32_t kNbS = G::kRxSBufs;
-    // this warp's region: row `lane` of it in the receive and the staging buffers
-    const uint32_t rxs_me = smem_u32(smem + G::kOffRxS) + region * kRxSRegion + lane * 128;
-    const uint32_t txs_me = smem_u32(smem + G::kOffTxS) + region * kRxSRegion + lane * 128;
-    const uint32_t rxp_me = smem_u32(smem + G::kOffRxP) + region * kRxPRegion + lane * 64;
-    const uint32_t txp_me = smem_u32(smem + G::kOffTxP) + region * kRxPRegion + lane * 64;
-    const uint32_t alpha_off = kRxPAlpha + (quad & 1) * 128;   // this quarter's 32 rescale factors
-    const uint32_t alpha_me = smem_u32(smem + G::kOffRxP) + alpha_off + lane * 4;
-    // 16-byte pieces of a lane's row are XOR-swizzled so that 8 consecutive lanes hit
-    // distinct banks: partial scores 128 B per row, probabilities 64 B per row
-    auto s_piece = [&](int c) { return (uint32_t)((c ^ (lane & 7)) << 4); };
-    auto p_piece = [&](int c) { return (uint32_t)((c ^ ((lane >> 1) & 3)) << 4); };
+    // Exchange regions: quarter q of every buffer holds 16 rows; a row is 64 fp32 scores
+    // (256 B) or 64 bf16 probabilities (128 B). Own warp q of one CTA and peer warp q + 4
+    // of the other fill / drain region q. 16-byte pieces of a row are XOR-swizzled by the
+    // row so that 8 consecutive rows hit distinct banks.
+    const uint32_t s_row = quad * kRxSRegion + rr * 256;
+    const uint32_t p_row = quad * kRxPRegion + rr * 128;
+    auto piece = [&](int c) { return (uint32_t)((c ^ (rr & 7)) << 4); };
+    const uint32_t rxs = smem_u32(smem + G::kOffRxS), txs = smem_u32(smem + G::kOffTxS);
+    const uint32_t rxp = smem_u32(smem + G::kOffRxP), txp = smem_u32(smem + G::kOffTxP);
+    const uint32_t alpha_off = kRxPAlpha + orow * 4;
     const int grow = rg * kRows + row;
     const bool valid_row = grow < a.rows;
     const int s_idx = valid_row ? grow / a.H : 0;
@@ -473,40 +476,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
     // PV(j) done. Valid while PV(j - 2) is complete and PV(j + 2) cannot be (its P is
     // not written yet): callers only wait for PVs of the current segment, in order.
     auto wait_pv = [&](uint32_t j) { return wait_local(smem_u32(&ctl.pv_done[j & 1]), (j >> 1) & 1); };
-    // O rows of this warp's lanes, its 128 columns, times alpha (all earlier PVs complete)
+    // O row of this thread (columns [128 hf, +128) of the CTA's 256) times alpha; all
+    // earlier PVs complete
     auto rescale_o = [&](float alpha) {
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         uint32_t v[16];
-        const uint32_t ta = tmem + lane_off + kTmemO + 128 * half + 16 * c;
-        tmem_ld16(ta, v);
+        const uint32_t ta = tmem + lane_off + kTmemO + 16 * c;
+        tmem_ld16x2<128>(ta, v);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-        tmem_st16(ta, v);
+        tmem_st16x2<128>(ta, v);
       }
       tmem_wait_st();
     };
-    // this warp's 32 partial-score columns of the current tile, out of TMEM
+    // this thread's 32 partial-score columns of the current tile, out of TMEM
     auto load_s = [&](uint32_t gt, uint32_t* sv) {
       if (!wait_local(smem_u32(&ctl.s_full), gt & 1)) return false;
       tc_fence_after();
-      tmem_ld16(tmem + lane_off + kTmemS + 32 * half, sv);
-      tmem_ld16(tmem + lane_off + kTmemS + 32 * half + 16, sv + 16);
+      tmem_ld16x2<32>(tmem + lane_off + kTmemS, sv);
+      tmem_ld16x2<32>(tmem + lane_off + kTmemS + 16, sv + 16);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(smem_u32(&ctl.s_empty));
       return true;
     };
     while (ok && it.next(sg)) {
-      // this segment's absorbed query, latent half of this CTA, into TMEM (all 128 rows)
+      // this segment's absorbed query, latent half of this CTA, into TMEM (the warp's 16 rows)
       ok = wait_local(smem_u32(&ctl.q_empty), (seg & 1) ^ 1);
       if (!ok) break;
       {
         uint32_t qv[64];
         const uint4* src = reinterpret_cast<const uint4*>((const uint16_t*)a.q_lat +
                                                          ((size_t)sg.b * a.rows + (valid_row ? grow : 0)) * kR +
-                                                         256 * rank + 128 * half);
+                                                         256 * rank + 128 * hf);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const uint4 v = valid_row ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
@@ -516,14 +520,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
           qv[4 * i + 3] = v.w;
         }
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_st16(tmem + lane_off + kTmemQ + 64 * half + 16 * c, qv + 16 * c);
+        for (int c = 0; c < 4; ++c) tmem_st16x2<64>(tmem + lane_off + kTmemQ + 16 * c, qv + 16 * c);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(smem_u32(&ctl.q_full));
       }
       const int n = sg.tile_end - sg.tile_begin;
       const int last_tile = (sg.Lc + kBS - 1) / kBS - 1;
-      float m_run = -INFINITY, l_run = 0.f;   // own rows: running maximum (log2 units) and sum
+      float m_run = -INFINITY, l_run = 0.f;   // own rows: running maximum (log2 units), this thread's sum
       if (own) {
         int n_row = valid_row ? (a.causal ? sg.Lc - a.Sq + 1 + s_idx : sg.Lc) : 0;
         if (n_row < 0) n_row = 0;
@@ -537,23 +541,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
           const uint32_t bs = gt % kNbS;
           ok = wait_peer(smem_u32(&ctl.rxs_full[bs]), (gt / kNbS) & 1);
           if (!ok) break;
-          const uint32_t rx = rxs_me + bs * kRxSBytes;
+          const uint32_t rx = rxs + bs * kRxSBytes + s_row;
           float x[32];
           float mh = -INFINITY;
-          const int valid = min(max(n_row - tile * kBS - 32 * half, 0), 32);   // of my 32 columns
+          const int valid = min(max(n_row - tile * kBS - 32 * hf, 0), 32);   // of my 32 columns
           const float4* cs = nullptr;   // FP8: token scales of my columns
           if constexpr (kFp8) {
             const uint32_t stg = gt % kStages;
             int dummy = 0;
             mbar_wait<false>(smem_u32(&ctl.kv_ready[stg]), (gt / kStages) & 1, &dummy, timeout_ns);
-            cs = reinterpret_cast<const float4*>(smem + kOffKv + stg * kStageBytes + G::kOffScale + 128 * half);
+            cs = reinterpret_cast<const float4*>(smem + kOffKv + stg * kStageBytes + G::kOffScale + 128 * hf);
           }
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint4 v;
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                         : "r"(rx + s_piece(c)));
+                         : "r"(rx + piece(8 * hf + c)));
             const float r4[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
                                  __uint_as_float(v.w)};
             float c4[4] = {1.f, 1.f, 1.f, 1.f};
@@ -572,15 +576,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
               mh = fmaxf(mh, x[k]);
             }
           }
-          ctl.mbuf[b][half][orow] = mh;   // depends on every value read from the receive buffer
+          const float mt = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));   // depends on every value read
           __syncwarp();
           // the peer may refill our region of buffer bs (tile gt + kNbS)
           if (lane == 0) mbar_arrive_remote_cta(mapa(smem_u32(&ctl.txs_ok[bs]), peer));
           if (leader) mbar_arrive_expect_tx(smem_u32(&ctl.rxs_full[bs]), kRxSBytes);
-          mbar_arrive(smem_u32(&ctl.mx[quad & 1]));
-          ok = wait_local(smem_u32(&ctl.mx[quad & 1]), gt & 1);
-          if (!ok) break;
-          const float mt = fmaxf(ctl.mbuf[b][0][orow], ctl.mbuf[b][1][orow]);
           // ---- exponentials, P into TMEM and to the peer
           const bool grow_max = mt > m_run + kRescaleThreshold;
           const bool rescale = grow_max && m_run != -INFINITY;
@@ -628,34 +628,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
               pk[k >> 1] = pack_bf16x2(p0, p1);
           }
           l_run += psum;
-          tmem_st16(tmem + lane_off + kTmemP + 32 * b + 16 * half, pk);
+          tmem_st16x2<16>(tmem + lane_off + kTmemP + 32 * b, pk);
           // stage the P row (and the rescale factor) like the peer's receive buffer; our
           // previous copy out of the staging region must have finished reading it
           if (lane == 0) bulk_wait_group_read<0>();
           __syncwarp();
 #pragma unroll
           for (int c = 0; c < 4; ++c)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(txp_me + p_piece(c)), "r"(pk[4 * c]),
-                         "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(txp + p_row + piece(4 * hf + c)),
+                         "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
                          : "memory");
-          if (half == 0)
-            asm volatile("st.shared.f32 [%0], %1;" ::"r"(smem_u32(smem + G::kOffTxP) + alpha_off + lane * 4),
-                         "f"(alpha)
-                         : "memory");
+          if (hf == 0)
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(txp + alpha_off), "f"(alpha) : "memory");
           fence_proxy_async_smem();
           // the peer's receive buffer is free once it has read tile gt - 1
           if (gt >= 1) {
             ok = wait_remote_arrival(smem_u32(&ctl.txp_ok), (gt - 1) & 1);
             if (!ok) break;
           }
+          __syncwarp();
           if (lane == 0) {
             const uint32_t bar = mapa(smem_u32(&ctl.rxp_full), peer);
-            const uint32_t rbase = region * kRxPRegion;
-            bulk_copy_to_peer(mapa(smem_u32(smem + G::kOffRxP) + rbase, peer), smem_u32(smem + G::kOffTxP) + rbase,
-                              kRxPRegion, bar);
-            if (half == 0)
-              bulk_copy_to_peer(mapa(smem_u32(smem + G::kOffRxP) + alpha_off, peer),
-                                smem_u32(smem + G::kOffTxP) + alpha_off, 128, bar);
+            bulk_copy_to_peer(mapa(rxp + quad * kRxPRegion, peer), txp + quad * kRxPRegion, kRxPRegion, bar);
+            bulk_copy_to_peer(mapa(rxp + kRxPAlpha + quad * 64, peer), txp + kRxPAlpha + quad * 64, 64, bar);
             bulk_commit_group();
           }
           // Slots past the sequence end in its last block may hold anything (NaN): zero
@@ -668,8 +663,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
                              timeout_ns);
             uint8_t* base = smem + kOffKv + stg * kStageBytes;
             const int per_chunk = (kBS - tail) * 8;          // 16-byte pieces per chunk
-            const int t0 = (quad & 1) * 32 + half * 64 + lane;   // 0..127 over the own warps
-            for (int i = t0; i < 4 * per_chunk; i += 128) {
+            for (int i = threadIdx.x; i < 4 * per_chunk; i += 128) {   // the 4 own warps
               const int chunk = i / per_chunk, rem = i % per_chunk;
               *reinterpret_cast<uint4*>(base + chunk * kKvLatChunk + (tail + rem / 8) * 128 + (rem % 8) * 16) =
                   make_uint4(0u, 0u, 0u, 0u);
@@ -681,9 +675,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
           mbar_arrive(smem_u32(&ctl.p_full[b]));
         }
       } else {
-        // Peer quarters: two in-order streams served as they become ready -- ship the
-        // partial scores of each tile to the peer, and take the peer's P rows of each tile
-        // into TMEM. Lane 0 polls, the warp follows its choice.
+        // Peer lanes: two in-order streams served as they become ready -- ship the partial
+        // scores of each tile to the peer, and take the peer's P rows of each tile into
+        // TMEM. Lane 0 polls, the warp follows its choice.
         int ship = 0, recv = 0;   // next segment-local tile of each stream
         uint32_t spins = 0;
         uint64_t t_idle = 0;
@@ -714,8 +708,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
             __syncwarp();
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(txs_me + s_piece(c)), "r"(sv[4 * c]),
-                           "r"(sv[4 * c + 1]), "r"(sv[4 * c + 2]), "r"(sv[4 * c + 3])
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(txs + s_row + piece(8 * hf + c)),
+                           "r"(sv[4 * c]), "r"(sv[4 * c + 1]), "r"(sv[4 * c + 2]), "r"(sv[4 * c + 3])
                            : "memory");
             fence_proxy_async_smem();
             // the peer's receive buffer bs is free once it has read tile gt - kNbS
@@ -723,11 +717,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
               ok = wait_remote_arrival(smem_u32(&ctl.txs_ok[bs]), ((gt / kNbS) + 1) & 1);
               if (!ok) break;
             }
+            __syncwarp();
             if (lane == 0) {
-              const uint32_t rbase = region * kRxSRegion;
-              bulk_copy_to_peer(mapa(smem_u32(smem + G::kOffRxS) + bs * kRxSBytes + rbase, peer),
-                                smem_u32(smem + G::kOffTxS) + rbase, kRxSRegion,
-                                mapa(smem_u32(&ctl.rxs_full[bs]), peer));
+              bulk_copy_to_peer(mapa(rxs + bs * kRxSBytes + quad * kRxSRegion, peer), txs + quad * kRxSRegion,
+                                kRxSRegion, mapa(smem_u32(&ctl.rxs_full[bs]), peer));
               bulk_commit_group();
             }
             ++ship;
@@ -736,14 +729,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
             ok = wait_peer(smem_u32(&ctl.rxp_full), gp & 1);   // completes at once
             if (!ok) break;
             uint32_t pk[16];
-            const uint32_t rx = rxp_me;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
               asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                            : "=r"(pk[4 * c]), "=r"(pk[4 * c + 1]), "=r"(pk[4 * c + 2]), "=r"(pk[4 * c + 3])
-                           : "r"(rx + p_piece(c)));
+                           : "r"(rxp + p_row + piece(4 * hf + c)));
             float alpha;
-            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(alpha) : "r"(alpha_me));
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(alpha) : "r"(rxp + alpha_off));
             if (recv >= 2) {   // P slot b held tile gp - 2 of this segment
               ok = wait_pv(gp - 2);
               if (!ok) break;
@@ -756,7 +748,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
               tc_fence_after();
               rescale_o(alpha);
             }
-            tmem_st16(tmem + lane_off + kTmemP + 32 * b + 16 * half, pk);   // consumes the loaded rows
+            tmem_st16x2<16>(tmem + lane_off + kTmemP + 32 * b, pk);   // consumes the loaded rows
             __syncwarp();
             if (lane == 0) mbar_arrive_remote_cta(mapa(smem_u32(&ctl.txp_ok), peer));
             if (leader) mbar_arrive_expect_tx(smem_u32(&ctl.rxp_full), kRxPBytes);   // tile gp + 1
@@ -777,12 +769,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
       tc_fence_after();
       float l_tot;
       if (own) {
-        ctl.lbuf[half][orow] = l_run;
-        mbar_arrive(smem_u32(&ctl.lx[quad & 1]));
-        ok = wait_local(smem_u32(&ctl.lx[quad & 1]), seg & 1);
-        if (!ok) break;
-        l_tot = ctl.lbuf[0][orow] + ctl.lbuf[1][orow];
-        if (half == 0)
+        l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+        if (hf == 0)
           st_async_b32(mapa(smem_u32(&ctl.lrx[seg & 1][orow]), peer), __float_as_uint(l_tot),
                        mapa(smem_u32(&ctl.lrx_full[seg & 1]), peer));
       } else {
@@ -799,10 +787,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         uint32_t v[16];
-        tmem_ld16(tmem + lane_off + kTmemO + 128 * half + 16 * c, v);
+        tmem_ld16x2<128>(tmem + lane_off + kTmemO + 16 * c, v);
         tmem_wait_ld();
         if (!valid_row) continue;
-        const int ch = 256 * (int)rank + 128 * half + 16 * c;
+        const int ch = 256 * (int)rank + 128 * hf + 16 * c;
         if (direct && a.out_dtype == kBF16) {
           uint4 o0, o1;
           o0.x = pack_bf16x2(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv);
@@ -825,7 +813,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
                             __uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv);
         }
       }
-      if (own && half == 0 && valid_row) {
+      if (own && hf == 0 && valid_row) {
         const float lse_v = l_tot > 0.f ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
         if (direct)
           a.lse[qrow] = lse_v;
