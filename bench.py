@@ -18,6 +18,7 @@ the host instead, on one sequence per step.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -62,6 +63,33 @@ def load_peaks():
         return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
                     bf16_tflops_sustained=d.get("bf16_tflops_sustained"), source="measured")
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture of the tcgen05
+# decode kernel on a smaller batch of the same workload; profiles/) per cached token. A figure
+# only holds for the kernel sources it was taken on, keyed here by their SHA-256 prefix; for
+# any other source the bench reports traffic as null.
+MEASURED_TRAFFIC = {
+    "d6dd6f34957f5978": {"deepseek_v3": (304.108032e6 + 4.895744e6) / 262144,
+                 "fp8_cache": (169.811968e6 + 4.268544e6) / 262144},
+}
+KERNEL_SOURCES = ("mla_tc.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.h", "mla_tc.h")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "head_latent_attention_split_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(wl, model, kernel):
+    """Per-launch DRAM bytes of the decode kernel scaled from the ncu capture, or None."""
+    if kernel != "tcgen05":
+        return None
+    per_tok = MEASURED_TRAFFIC.get(kernel_source_hash(), {}).get(wl.name)
+    return None if per_tok is None else per_tok * model["tokens"]
 
 
 def work_model(inp):
@@ -340,7 +368,7 @@ def main():
             steps_per_s=K / sec,
             tokens_per_s=world * K * wl.B * wl.Sq / sec,
             roofline=dict(bound=bound, achieved=achieved, peak=peak, unit=unit, frac=achieved / peak,
-                          traffic=None),
+                          traffic=measured_traffic(wl, model, kernel)),
             roofline_detail=dict(
                 kernel=f"decode ({kernel})", decode_ms=1e3 * dec_s, combine_ms=statistics.mean(comb_ms),
                 algorithmic_bytes=model["bytes"], algorithmic_flops=model["flops"],
