@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--op", default="decode", choices=["decode", "append"],
+                    help="decode: the decode step (default); append: the paged cache append of the step's new tokens")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller profiling captures only)")
     return ap.parse_args()
@@ -220,6 +222,60 @@ def reference_arm(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def append_arm(args, rank, local):
+    """Time mla_cache_append for the workload's B x Sq new tokens (rotated RoPE keys)."""
+    import torch
+    import head_latent_attention_split_b200 as mla
+    wl = W.BY_NAME[args.workload]
+    if args.batch:
+        wl = wl.with_(B=args.batch)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    lens = np.asarray(W.resolve_seq_lens(wl), np.int32)
+    bs = wl.block_size
+    mb = int((lens.max() + bs - 1) // bs)
+    nb = wl.B * mb
+    bt = torch.randperm(nb, dtype=torch.int32, device=dev).reshape(wl.B, mb)
+    sl = torch.from_numpy(lens).to(dev)
+    g = torch.Generator(device=dev).manual_seed(1000 + W.WORKLOADS.index(W.BY_NAME[args.workload]))
+    c = torch.randn((wl.B, wl.Sq, wl.r), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((wl.B, wl.Sq, wl.d_r), generator=g, device=dev).to(torch.bfloat16)
+    fp8 = wl.cache_dtype == W.E4M3
+    if fp8:
+        cache = torch.zeros((nb, bs, wl.r), dtype=torch.uint8, device=dev)
+        kr = torch.zeros((nb, bs, wl.d_r), dtype=torch.bfloat16, device=dev)
+        sc = torch.zeros((nb, bs), dtype=torch.float32, device=dev)
+    else:
+        cache = torch.zeros((nb, bs, wl.r + wl.d_r), dtype=torch.bfloat16, device=dev)
+        kr = sc = None
+    run = lambda: mla.cache_append(c, k, cache, bt, sl, k_rope_cache=kr, kv_scale=sc, rope=True)  # noqa: E731
+    for _ in range(max(args.warmup, 3)):
+        run()
+    torch.cuda.synchronize()
+    assert mla.device_status() == 0
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(args.steps):
+        run()
+    ev[1].record()
+    torch.cuda.synchronize()
+    us = 1e3 * ev[0].elapsed_time(ev[1]) / args.steps
+    ntok = wl.B * wl.Sq
+    bytes_ = ntok * ((wl.r + wl.d_r) * 2 + W.cache_bytes_per_token(wl.r, wl.d_r, wl.cache_dtype))
+    peaks = load_peaks()
+    gbs = bytes_ / (us * 1e-6) / 1e9
+    if rank == 0:
+        print(json.dumps(dict(
+            metric="paged cache append GB/s (new tokens read + cache slots written)", value=gbs, unit="GB/s",
+            n_gpus=1, steps=args.steps, warmup=max(args.warmup, 3), us_per_call=us, higher_is_better=True,
+            dtype="bf16->" + W.DTYPE_NAMES[wl.cache_dtype], data="synthetic",
+            config=dict(workload=wl.name, op="append", B=wl.B, Sq=wl.Sq, r=wl.r, d_r=wl.d_r, rope=True,
+                        new_tokens=ntok, bytes_per_call=bytes_),
+            roofline=dict(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s", frac=gbs / peaks["hbm_gbs"],
+                          traffic=None, note="launch-latency bound: one call moves only bytes_per_call"),
+            gpu_launches=args.steps)), flush=True)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -227,6 +283,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         reference_arm(args, rank)
+        return
+    if args.op == "append":
+        append_arm(args, rank, local)
         return
 
     import torch

@@ -71,3 +71,20 @@ def decode_host_io(q_lat_host, q_rope_host, kv_cache, block_table_host, seq_lens
     _b.mla_decode_host_io(p, q_lat_host, q_rope_host, kv_cache, k_rope_cache, kv_scale, block_table_host,
                           seq_lens_host, out_host, lse_host, workspace, stream=stream)
     return out_host, lse_host
+
+
+def cache_append(c_new, k_rope_new, kv_cache, block_table, seq_lens, k_rope_cache=None, kv_scale=None,
+                 rope=False, rope_base=10000.0, stream=None):
+    """Write the Sq new tokens of each sequence into the paged cache (see mla_cache_append).
+
+    c_new [B, Sq, r] and k_rope_new [B, Sq, d_r] (float32 for an f32 cache, bf16 otherwise);
+    kv_cache [num_blocks, block_size, r + d_r] (f32 / bf16), or e4m3 codes
+    [num_blocks, block_size, r] (uint8) with k_rope_cache bf16 [num_blocks, block_size, d_r]
+    and kv_scale float32 [num_blocks, block_size]. Token s of sequence b lands at position
+    seq_lens[b] - Sq + s. With rope, the RoPE key is rotated for that position first.
+    """
+    B, Sq, r = c_new.shape
+    d_r = k_rope_new.shape[-1] if k_rope_new is not None else 0
+    p = _b.make_append_params(B, Sq, r, d_r, kv_cache.shape[1], kv_cache.shape[0], block_table.shape[1],
+                              _dtype_code(c_new, "c_new"), _dtype_code(kv_cache, "kv_cache"), rope, rope_base)
+    _b.mla_cache_append(p, c_new, k_rope_new, kv_cache, k_rope_cache, kv_scale, block_table, seq_lens, stream=stream)

@@ -26,7 +26,7 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "M
 EXPORTED = ("mla_decode_workspace_size", "mla_decode_resolve", "mla_decode", "mla_decode_timed",
             "mla_decode_host_io_workspace_size", "mla_decode_host_io", "mla_plan_host", "mla_plan_probe",
             "mla_get_device_status", "mla_status_string", "mla_abi_version", "mla_decode_noalloc",
-            "mla_decode_noalloc_max_workspace")
+            "mla_decode_noalloc_max_workspace", "mla_cache_append")
 
 
 class MlaError(RuntimeError):
@@ -42,6 +42,15 @@ class Params(ctypes.Structure):
         "max_blocks_per_seq", "q_dtype", "cache_dtype", "out_dtype", "causal")] + [
         ("softmax_scale", ctypes.c_float), ("num_workers", ctypes.c_int32), ("kernel", ctypes.c_int32),
         ("reserved", ctypes.c_int32)]
+
+
+class AppendParams(ctypes.Structure):
+    """mla_append_params_t."""
+    _fields_ = [("batch", ctypes.c_int32), ("q_len", ctypes.c_int32), ("kv_rank", ctypes.c_int32),
+                ("rope_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
+                ("max_blocks_per_seq", ctypes.c_int32), ("in_dtype", ctypes.c_int32),
+                ("cache_dtype", ctypes.c_int32), ("rope", ctypes.c_int32), ("rope_base", ctypes.c_float),
+                ("reserved", ctypes.c_int32)]
 
 
 def _load():
@@ -66,6 +75,7 @@ def _load():
     L.mla_status_string.argtypes = [ctypes.c_int32]
     L.mla_status_string.restype = ctypes.c_char_p
     L.mla_abi_version.argtypes = []
+    L.mla_cache_append.argtypes = [ctypes.POINTER(AppendParams), vp, vp, vp, vp, vp, vp, vp, vp]
     for name in EXPORTED:
         if not hasattr(L, name):
             raise ImportError(f"{LIB_PATH} lacks {name}: rebuild it")
@@ -233,3 +243,21 @@ def status_string(st: int) -> str:
 
 def abi_version() -> int:
     return lib.mla_abi_version()
+
+
+def make_append_params(B, Sq, r, d_r, block_size, num_blocks, max_blocks_per_seq, in_dtype, cache_dtype,
+                       rope=False, rope_base=10000.0) -> AppendParams:
+    return AppendParams(batch=B, q_len=Sq, kv_rank=r, rope_dim=d_r, block_size=block_size, num_blocks=num_blocks,
+                        max_blocks_per_seq=max_blocks_per_seq, in_dtype=in_dtype, cache_dtype=cache_dtype,
+                        rope=int(bool(rope)), rope_base=float(rope_base), reserved=0)
+
+
+def mla_cache_append(p: AppendParams, c_new, k_rope_new, kv_cache, k_rope_cache, kv_scale, block_table, seq_lens,
+                     stream=None, check=True) -> int:
+    """Raw C-ABI call of the paged cache append (device tensors or integer addresses)."""
+    st = lib.mla_cache_append(ctypes.byref(p), _addr(c_new), _addr(k_rope_new), _addr(kv_cache),
+                              _addr(k_rope_cache), _addr(kv_scale), _addr(block_table), _addr(seq_lens),
+                              _stream(stream))
+    if check:
+        _check(st, "mla_cache_append")
+    return st

@@ -364,6 +364,51 @@ mla_status_t mla_plan_probe(const mla_decode_params_t* p, const int32_t* block_t
                                                                                                  : MLA_ERR_CUDA;
 }
 
+mla_status_t mla_cache_append(const mla_append_params_t* p, const void* c_new, const void* k_rope_new,
+                              void* kv_cache, void* k_rope_cache, float* kv_scale, const int32_t* block_table,
+                              const int32_t* seq_lens, void* stream) {
+  if (!p) return MLA_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->q_len < 1 || p->kv_rank < 1 || p->rope_dim < 0 || p->block_size < 1 ||
+      p->num_blocks < 0 || p->max_blocks_per_seq < 1 || p->reserved != 0 || (p->rope != 0 && p->rope != 1))
+    return MLA_ERR_INVALID_ARG;
+  if (p->batch > 0 && p->num_blocks < 1) return MLA_ERR_INVALID_ARG;
+  const bool pair_ok = (p->in_dtype == MLA_DTYPE_F32 && p->cache_dtype == MLA_DTYPE_F32) ||
+                       (p->in_dtype == MLA_DTYPE_BF16 &&
+                        (p->cache_dtype == MLA_DTYPE_BF16 || p->cache_dtype == MLA_DTYPE_E4M3));
+  if (!pair_ok) return MLA_ERR_INVALID_ARG;
+  if (p->cache_dtype == MLA_DTYPE_E4M3 && (p->kv_rank % 2 != 0 || !k_rope_cache || !kv_scale))
+    return MLA_ERR_INVALID_ARG;
+  if (p->rope && (p->rope_dim % 2 != 0 || !std::isfinite(p->rope_base) || !(p->rope_base > 0.f)))
+    return MLA_ERR_INVALID_ARG;
+  if (p->batch == 0) return MLA_OK;
+  if (!c_new || !kv_cache || !block_table || !seq_lens || (p->rope_dim > 0 && !k_rope_new))
+    return MLA_ERR_INVALID_ARG;
+  if ((int64_t)p->max_blocks_per_seq * p->block_size > (1ll << 30)) return MLA_ERR_UNSUPPORTED;
+  int* status = status_word(current_device());
+  if (!status) return MLA_ERR_CUDA;
+  mla::AppendArgs a{};
+  a.B = p->batch;
+  a.Sq = p->q_len;
+  a.r = p->kv_rank;
+  a.d_r = p->rope_dim;
+  a.bs = p->block_size;
+  a.num_blocks = p->num_blocks;
+  a.max_blocks = p->max_blocks_per_seq;
+  a.in_dtype = p->in_dtype;
+  a.cache_dtype = p->cache_dtype;
+  a.rope = p->rope;
+  a.rope_base = p->rope_base;
+  a.c_new = c_new;
+  a.k_new = k_rope_new;
+  a.cache = kv_cache;
+  a.k_rope = (uint16_t*)k_rope_cache;
+  a.kv_scale = kv_scale;
+  a.block_table = block_table;
+  a.seq_lens = seq_lens;
+  a.status = status;
+  return mla::launch_cache_append(a, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 mla_status_t mla_get_device_status(void* stream, int32_t* device_status) {
   if (!device_status) return MLA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MLA_ERR_CUDA;

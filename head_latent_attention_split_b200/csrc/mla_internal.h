@@ -71,4 +71,20 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_plan_probe(const DecodeArgs& a, int32_t* token_slot, int32_t* token_worker,
                               cudaStream_t s);
 
+// Arguments of the paged cache append kernel (mla_append.cu).
+struct AppendArgs {
+  int B, Sq, r, d_r, bs, num_blocks, max_blocks;
+  int in_dtype, cache_dtype, rope;
+  float rope_base;
+  const void* c_new;           // [B, Sq, r] in_dtype
+  const void* k_new;           // [B, Sq, d_r] in_dtype
+  void* cache;                 // F32/BF16: [nb, bs, r + d_r]; E4M3: codes [nb, bs, r]
+  uint16_t* k_rope;            // E4M3 only: bf16 [nb, bs, d_r]
+  float* kv_scale;             // E4M3 only: [nb, bs]
+  const int32_t* block_table;  // [B, max_blocks]
+  const int32_t* seq_lens;     // [B]
+  int* status;
+};
+cudaError_t launch_cache_append(const AppendArgs& a, cudaStream_t s);
+
 }  // namespace mla

@@ -203,6 +203,55 @@ mla_status_t mla_get_device_status(void* stream, int32_t* device_status);
 /* Static, human-readable name of a status code. */
 const char* mla_status_string(int32_t status);
 
+/* ------------------------------------------------------------------ cache append
+ *
+ * Writes the latent and RoPE key of the Sq new tokens of every sequence into the paged
+ * cache that mla_decode reads ("TransMLA: Multi-Head Latent Attention Is All You Need",
+ * sec. 3.4.5: the cache holds one latent c and one decoupled RoPE key kR per token, and
+ * the RoPE key is recomputed for the new token at its position; the "Watching the fusion
+ * actually fail, on numbers" passage of the TransMLA & Sparse Latent Attention lesson shows
+ * the position rotation R(t) on a two-dimensional toy).
+ *
+ * Token s of sequence b has logical position pos = seq_lens[b] - Sq + s (the Sq new tokens
+ * are the last Sq of seq_lens[b], the convention of mla_decode's causal mode) and goes to
+ * physical block block_table[b][pos / block_size], slot pos % block_size.
+ *   - in_dtype MLA_F32 -> cache_dtype MLA_F32, or MLA_BF16 -> MLA_BF16: the values are stored
+ *     as given ([num_blocks][block_size][r + d_r]).
+ *   - in_dtype MLA_BF16 -> cache_dtype MLA_E4M3: the latent is quantised per token:
+ *     scale = max_k |c_k| / 448 (fp32 division), code_k = e4m3(c_k / scale) (fp32 division,
+ *     round to nearest even, saturated to +-448; OCP FP8 e4m3, no infinities); scale 0 (an
+ *     all-zero latent) stores zero codes. Codes go to kv_cache [num_blocks][block_size][r],
+ *     the scale to kv_scale [num_blocks][block_size], the bf16 RoPE key to k_rope_cache
+ *     [num_blocks][block_size][d_r].
+ *   - rope != 0: the RoPE key is rotated before it is stored: pairs (x[2i], x[2i+1]) turn by
+ *     pos * theta_i with theta_i = rope_base^(-2i / d_r) (angle and rotation in fp64, result
+ *     rounded to the cache type). rope == 0 stores k_rope_new as given (already rotated).
+ *
+ * c_new [B, Sq, r] and k_rope_new [B, Sq, d_r] have type in_dtype; all pointers are device
+ * pointers; the call is asynchronous on `stream` and allocates nothing. Argument errors
+ * return at once without a launch. A token whose position is negative or past the block
+ * table raises MLA_ERR_BAD_SEQ_LEN, one whose block id is out of range MLA_ERR_BAD_BLOCK_ID
+ * (sticky device status word, read with mla_get_device_status); such tokens are not
+ * written. Tokens of different sequences must map to different slots. */
+typedef struct {
+  int32_t batch;               /* B */
+  int32_t q_len;               /* Sq: new tokens per sequence */
+  int32_t kv_rank;             /* r */
+  int32_t rope_dim;            /* d_r (even when rope != 0) */
+  int32_t block_size;
+  int32_t num_blocks;
+  int32_t max_blocks_per_seq;  /* row stride of block_table */
+  int32_t in_dtype;            /* mla_dtype_t of c_new and k_rope_new */
+  int32_t cache_dtype;         /* mla_dtype_t of the cache */
+  int32_t rope;                /* 0: store k_rope_new as given; 1: rotate it first */
+  float rope_base;             /* theta base of the rotation, e.g. 10000 */
+  int32_t reserved;            /* must be 0 */
+} mla_append_params_t;
+
+mla_status_t mla_cache_append(const mla_append_params_t* params, const void* c_new, const void* k_rope_new,
+                              void* kv_cache, void* k_rope_cache, float* kv_scale, const int32_t* block_table,
+                              const int32_t* seq_lens, void* stream);
+
 /* MLA_DECODE_ABI_VERSION of the loaded library. */
 int32_t mla_abi_version(void);
 

@@ -77,6 +77,12 @@ def lib():
         L.mla_oracle_bf16_to_double.restype = ctypes.c_double
         L.mla_oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
         L.mla_oracle_e4m3_to_double.restype = ctypes.c_double
+        L.mla_oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.mla_oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.mla_oracle_e4m3_encode_n.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64]
+        L.mla_oracle_e4m3_encode_n.restype = None
+        L.mla_oracle_cache_append.argtypes = [ctypes.c_int] * 10 + [ctypes.c_double] + [ctypes.c_void_p] * 7
+        L.mla_oracle_cache_append.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -213,3 +219,35 @@ def decode_rows_inputs(inp: dict, rows, nthreads=0):
     return decode_rows(rows, inp["q_lat"], inp["q_rope"], inp["kv_cache"], inp["block_table"],
                        inp["seq_lens"], w.scale, w.causal, inp.get("k_rope_cache"),
                        inp.get("kv_scale"), w.block_size, nthreads=nthreads)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """fp32 values -> OCP e4m3 codes (nearest, ties to even, saturated to +-448)."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    codes = np.empty(x.shape, dtype=np.uint8)
+    lib().mla_oracle_e4m3_encode_n(x.ctypes.data, codes.ctypes.data, x.size)
+    return codes
+
+
+def cache_append(*, B, Sq, r, d_r, block_size, num_blocks, max_blocks_per_seq, in_dtype, cache_dtype,
+                 c_new, k_new, kv_cache, block_table, seq_lens, k_rope_cache=None, kv_scale=None,
+                 rope=False, rope_base=10000.0) -> int:
+    """Write the new tokens into the paged cache arrays in place (see mla_oracle.c).
+
+    c_new / k_new: [B, Sq, r] / [B, Sq, d_r] as float32 (in_dtype F32) or bf16 bit
+    patterns in uint16 (BF16). kv_cache: float32 / uint16 [num_blocks, bs, r + d_r], or
+    uint8 codes [num_blocks, bs, r] with k_rope_cache uint16 [num_blocks, bs, d_r] and
+    kv_scale float32 [num_blocks, bs] for E4M3. Returns the oracle status (0 = ok).
+    """
+    c_new = np.ascontiguousarray(c_new)
+    k_new = np.ascontiguousarray(k_new)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    for a in (kv_cache, k_rope_cache, kv_scale):
+        if a is not None:
+            assert a.flags["C_CONTIGUOUS"]
+    ptr = lambda a: None if a is None else a.ctypes.data  # noqa: E731
+    return lib().mla_oracle_cache_append(
+        B, Sq, r, d_r, block_size, num_blocks, max_blocks_per_seq, in_dtype, cache_dtype, int(bool(rope)),
+        float(rope_base), c_new.ctypes.data, k_new.ctypes.data, kv_cache.ctypes.data, ptr(k_rope_cache),
+        ptr(kv_scale), bt.ctypes.data, sl.ctypes.data)

@@ -23,7 +23,8 @@
  *   Rows that see no token get out = 0 and lse = -inf.
  *
  * The softmax is the two-pass textbook form in fp64 (max, then sum of exponentials),
- * with every stored input decoded exactly to double first:
+ * with every stored input decoded exactly to double first (the cache append at the end
+ * of this file writes that cache):
  *   f32  -> double (exact), f64 as is,
  *   bf16 -> the fp32 whose upper 16 bits are the pattern (exact),
  *   e4m3 (OCP FP8: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no
@@ -304,4 +305,119 @@ void mla_oracle_merge(int n_parts, int n_rows, int r, const double* o_parts, con
     }
     lse[row] = L;
   }
+}
+
+/* ------------------------------------------------------------------ cache append
+ *
+ * The producer side of the cache the decode reads ("TransMLA: Multi-Head Latent
+ * Attention Is All You Need", sec. 3.4.5: one latent and one decoupled RoPE key per
+ * token; the RoPE key is rotated for the token's position, as the "Watching the fusion
+ * actually fail, on numbers" passage of the TransMLA & Sparse Latent Attention lesson
+ * shows with R(t) on a 2-D toy).
+ */
+
+/* fp32 -> OCP e4m3 code, round to nearest with ties to the even code, magnitudes above
+ * 448 saturate to 448, NaN -> 0x7F. Plain search over the 127 finite magnitudes. */
+uint8_t mla_oracle_e4m3_encode(float x) {
+  if (isnan(x)) return 0x7F;
+  const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  const double a = fabs((double)x);
+  int best = 0;
+  double best_err = INFINITY;
+  for (int c = 0; c <= 0x7E; ++c) {
+    const double err = fabs(mla_oracle_e4m3_to_double((uint8_t)c) - a);
+    if (err < best_err || (err == best_err && (c & 1) == 0)) {
+      best = c;
+      best_err = err;
+    }
+  }
+  return (uint8_t)(sign | best);
+}
+
+void mla_oracle_e4m3_encode_n(const float* x, uint8_t* codes, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) codes[i] = mla_oracle_e4m3_encode(x[i]);
+}
+
+/* fp32 -> bf16 bits, round to nearest even (finite inputs). */
+static uint16_t f32_to_bf16_rne(float f) {
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+/*
+ * For token s of sequence b (pos = seq_lens[b] - Sq + s, block block_table[b][pos / bs],
+ * slot pos % bs): store the latent (as given, or as e4m3 codes with the per-token scale
+ * max|c| / 448 computed in fp32 and codes e4m3(c / scale) of the fp32 quotient), and the
+ * RoPE key, rotated first when rope is set: pairs (x[2i], x[2i+1]) turn by
+ * pos * base^(-2i / d_r), in fp64, rounded to fp32 and then to the cache type.
+ * Tokens with a bad position or block id are skipped; the first such error is returned.
+ */
+int mla_oracle_cache_append(int B, int Sq, int r, int d_r, int bs, int num_blocks, int max_blocks,
+                            int in_dtype, int cache_dtype, int rope, double rope_base, const void* c_new,
+                            const void* k_new, void* cache, uint16_t* k_rope_cache, float* kv_scale,
+                            const int32_t* block_table, const int32_t* seq_lens) {
+  int err = OR_OK;
+  const int D = r + d_r;
+  for (int b = 0; b < B; ++b) {
+    for (int s = 0; s < Sq; ++s) {
+      const int64_t pos = (int64_t)seq_lens[b] - Sq + s;
+      if (pos < 0 || pos >= (int64_t)max_blocks * bs) {
+        if (!err) err = OR_ERR_SEQ_LEN;
+        continue;
+      }
+      const int32_t blk = block_table[(size_t)b * max_blocks + pos / bs];
+      if (blk < 0 || blk >= num_blocks) {
+        if (!err) err = OR_ERR_BLOCK_ID;
+        continue;
+      }
+      const size_t slot = (size_t)blk * bs + (size_t)(pos % bs);
+      const size_t row = (size_t)b * Sq + s;
+      /* latent */
+      if (cache_dtype == OR_E4M3) {
+        const uint16_t* c = (const uint16_t*)c_new + row * r;
+        float amax = 0.f;
+        for (int k = 0; k < r; ++k) {
+          const float v = (float)mla_oracle_bf16_to_double(c[k]);
+          if (fabsf(v) > amax) amax = fabsf(v);
+        }
+        const float scale = amax / 448.0f;
+        uint8_t* codes = (uint8_t*)cache + slot * r;
+        for (int k = 0; k < r; ++k) {
+          const float v = (float)mla_oracle_bf16_to_double(c[k]);
+          codes[k] = mla_oracle_e4m3_encode(scale > 0.f ? v / scale : 0.f);
+        }
+        kv_scale[slot] = scale;
+      } else if (cache_dtype == OR_BF16) {
+        memcpy((uint16_t*)cache + slot * D, (const uint16_t*)c_new + row * r, (size_t)r * 2);
+      } else {
+        memcpy((float*)cache + slot * D, (const float*)c_new + row * r, (size_t)r * 4);
+      }
+      /* RoPE key */
+      for (int j = 0; j < d_r; ++j) {
+        double y;
+        const double x = load_elem(k_new, in_dtype, row * d_r + j);
+        if (rope) {
+          const int i = j / 2;
+          const double theta = pow(rope_base, -2.0 * i / d_r);
+          const double ang = (double)pos * theta;
+          const double x0 = load_elem(k_new, in_dtype, row * d_r + 2 * i);
+          const double x1 = load_elem(k_new, in_dtype, row * d_r + 2 * i + 1);
+          const double cs = cos(ang), sn = sin(ang);
+          y = (j % 2 == 0) ? x0 * cs - x1 * sn : x0 * sn + x1 * cs;
+        } else {
+          y = x;
+        }
+        const float yf = (float)y;
+        if (cache_dtype == OR_F32)
+          ((float*)cache)[slot * D + r + j] = yf;
+        else if (cache_dtype == OR_BF16)
+          ((uint16_t*)cache)[slot * D + r + j] = f32_to_bf16_rne(yf);
+        else
+          k_rope_cache[slot * d_r + j] = f32_to_bf16_rne(yf);
+      }
+    }
+  }
+  return err;
 }

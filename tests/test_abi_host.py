@@ -169,3 +169,35 @@ def test_plan_host_rejects_bad_lengths(m):
         m.plan_host(p, [65, 3])
     with pytest.raises(Exception):
         m.plan_host(p, [-1, 3])
+
+
+# ----------------------------------------------------------------------------- cache append
+def _append(m, stream=0, **kw):
+    from head_latent_attention_split_b200 import binding
+    args = dict(B=2, Sq=1, r=512, d_r=64, block_size=64, num_blocks=8, max_blocks_per_seq=4, in_dtype=1,
+                cache_dtype=1, rope=False, rope_base=10000.0)
+    ptrs = dict(c_new=FAKE, k_rope_new=FAKE, kv_cache=FAKE, k_rope_cache=None, kv_scale=None, block_table=FAKE,
+                seq_lens=FAKE)
+    for k in list(kw):
+        if k in ptrs:
+            ptrs[k] = kw.pop(k)
+    reserved = kw.pop("reserved", 0)
+    args.update(kw)
+    p = binding.make_append_params(**args)
+    p.reserved = reserved
+    return binding.mla_cache_append(p, stream=stream, check=False, **ptrs)
+
+
+@pytest.mark.parametrize("bad", [dict(Sq=0), dict(r=0), dict(d_r=-1), dict(block_size=0), dict(max_blocks_per_seq=0),
+                                 dict(num_blocks=0), dict(in_dtype=0), dict(in_dtype=2), dict(cache_dtype=0),
+                                 dict(in_dtype=0, cache_dtype=2), dict(reserved=1),
+                                 dict(cache_dtype=2, r=511, k_rope_cache=FAKE, kv_scale=FAKE),
+                                 dict(cache_dtype=2), dict(rope=True, d_r=63), dict(rope=True, rope_base=0.0),
+                                 dict(rope=True, rope_base=float("inf")), dict(c_new=None), dict(kv_cache=None),
+                                 dict(block_table=None), dict(seq_lens=None), dict(k_rope_new=None)])
+def test_append_rejects_bad_arguments_on_host(m, bad):
+    assert _append(m, **bad) == 1      # MLA_ERR_INVALID_ARG, nothing launched
+
+
+def test_append_batch_zero_is_a_noop(m):
+    assert _append(m, B=0, c_new=None, kv_cache=None, block_table=None, seq_lens=None) == 0
