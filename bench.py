@@ -51,8 +51,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--op", default="decode", choices=["decode", "append"],
-                    help="decode: the decode step (default); append: the paged cache append of the step's new tokens")
+    ap.add_argument("--op", default="decode", choices=["decode", "append", "absorb", "project"],
+                    help="decode: the decode step (default); append: the paged cache append of the step's new "
+                         "tokens; absorb / project: the per-head W^UK / W^UV products around the decode")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller profiling captures only)")
     return ap.parse_args()
@@ -276,6 +277,50 @@ def append_arm(args, rank, local):
             gpu_launches=args.steps)), flush=True)
 
 
+def head_gemm_arm(args, rank, local):
+    """Time the per-head GEMM of the workload's query rows: absorb (d_h = 128 -> r) or project (r -> d_v = 128)."""
+    import torch
+    import head_latent_attention_split_b200 as mla
+    wl = W.BY_NAME[args.workload]
+    if args.batch:
+        wl = wl.with_(B=args.batch)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    rows, H = wl.B * wl.Sq, wl.H
+    k, n = (128, wl.r) if args.op == "absorb" else (wl.r, 128)
+    g = torch.Generator(device=dev).manual_seed(7)
+    x = torch.randn((rows, H, k), generator=g, device=dev).to(torch.bfloat16)
+    w = (torch.randn((H, k, n), generator=g, device=dev) / math.sqrt(k)).to(torch.bfloat16)
+    y = torch.empty((rows, H, n), dtype=torch.bfloat16, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        mla.head_gemm(x, w, y)
+    torch.cuda.synchronize()
+    assert mla.device_status() == 0
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(args.steps):
+        mla.head_gemm(x, w, y)
+    ev[1].record()
+    torch.cuda.synchronize()
+    us = 1e3 * ev[0].elapsed_time(ev[1]) / args.steps
+    flops = 2.0 * rows * H * k * n
+    bytes_ = 2 * (rows * H * (k + n) + H * k * n)
+    peaks = load_peaks()
+    t_roof = max(bytes_ / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+    bound = "hbm" if bytes_ / (peaks["hbm_gbs"] * 1e9) >= flops / (peaks["bf16_tflops"] * 1e12) else "tensor"
+    achieved = bytes_ / (us * 1e-6) / 1e9 if bound == "hbm" else flops / (us * 1e-6) / 1e12
+    if rank == 0:
+        print(json.dumps(dict(
+            metric=f"per-head {'query absorption' if args.op == 'absorb' else 'output projection'} TFLOP/s",
+            value=flops / (us * 1e-6) / 1e12, unit="TFLOP/s", n_gpus=1, steps=args.steps,
+            warmup=max(args.warmup, 3), us_per_call=us, higher_is_better=True, dtype="bf16", data="synthetic",
+            config=dict(workload=wl.name, op=args.op, rows=rows, H=H, k=k, n=n),
+            roofline=dict(bound=bound, achieved=achieved, peak=peaks["hbm_gbs"] if bound == "hbm" else
+                          peaks["bf16_tflops"], unit="GB/s" if bound == "hbm" else "TFLOP/s",
+                          frac=t_roof / (us * 1e-6), traffic=None),
+            gpu_launches=args.steps)), flush=True)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -286,6 +331,9 @@ def main():
         return
     if args.op == "append":
         append_arm(args, rank, local)
+        return
+    if args.op in ("absorb", "project"):
+        head_gemm_arm(args, rank, local)
         return
 
     import torch

@@ -7,8 +7,8 @@ key and value. The kernels live in libmla_decode.so (C ABI: include/mla_decode.h
 this package is a thin binding over it.
 """
 from .binding import (BF16, E4M3, F32, KERNELS, AppendParams, MlaError, Params, abi_version,  # noqa: F401
-                      device_status, make_append_params, mla_cache_append,
+                      HeadGemmParams, device_status, make_append_params, mla_cache_append, mla_head_gemm,
                       host_io_workspace_size, make_params, mla_decode, mla_decode_host_io, mla_decode_timed, plan_host,
                       mla_decode_noalloc, noalloc_max_workspace,
                       plan_probe, resolve, status_string, workspace_size)
-from .api import cache_append, decode, decode_host_io, params_for  # noqa: F401
+from .api import cache_append, decode, decode_host_io, head_gemm, params_for  # noqa: F401

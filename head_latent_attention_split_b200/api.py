@@ -88,3 +88,21 @@ def cache_append(c_new, k_rope_new, kv_cache, block_table, seq_lens, k_rope_cach
     p = _b.make_append_params(B, Sq, r, d_r, kv_cache.shape[1], kv_cache.shape[0], block_table.shape[1],
                               _dtype_code(c_new, "c_new"), _dtype_code(kv_cache, "kv_cache"), rope, rope_base)
     _b.mla_cache_append(p, c_new, k_rope_new, kv_cache, k_rope_cache, kv_scale, block_table, seq_lens, stream=stream)
+
+
+def head_gemm(x, w, y=None, stream=None):
+    """y[m, h, :] = x[m, h, :] @ w[h] on the tensor cores (bf16 in and out, fp32 accumulation).
+
+    x [rows, H, k] (or [B, Sq, H, k]), w [H, k, n]; k and n multiples of 64. Query absorption:
+    head_gemm(q_nope, W_UK) -> q_lat; output projection: head_gemm(out, W_UV.transpose(1, 2)).
+    """
+    import torch
+    lead = x.shape[:-2]
+    H, k = x.shape[-2], x.shape[-1]
+    n = w.shape[-1]
+    rows = int(x.numel() // (H * k))
+    if y is None:
+        y = torch.empty((*lead, H, n), dtype=torch.bfloat16, device=x.device)
+    p = _b.HeadGemmParams(rows=rows, heads=H, k=k, n=n, reserved=0)
+    _b.mla_head_gemm(p, x, w, y, stream=stream)
+    return y

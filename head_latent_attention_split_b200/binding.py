@@ -26,7 +26,7 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "M
 EXPORTED = ("mla_decode_workspace_size", "mla_decode_resolve", "mla_decode", "mla_decode_timed",
             "mla_decode_host_io_workspace_size", "mla_decode_host_io", "mla_plan_host", "mla_plan_probe",
             "mla_get_device_status", "mla_status_string", "mla_abi_version", "mla_decode_noalloc",
-            "mla_decode_noalloc_max_workspace", "mla_cache_append")
+            "mla_decode_noalloc_max_workspace", "mla_cache_append", "mla_head_gemm")
 
 
 class MlaError(RuntimeError):
@@ -42,6 +42,12 @@ class Params(ctypes.Structure):
         "max_blocks_per_seq", "q_dtype", "cache_dtype", "out_dtype", "causal")] + [
         ("softmax_scale", ctypes.c_float), ("num_workers", ctypes.c_int32), ("kernel", ctypes.c_int32),
         ("reserved", ctypes.c_int32)]
+
+
+class HeadGemmParams(ctypes.Structure):
+    """mla_head_gemm_params_t."""
+    _fields_ = [("rows", ctypes.c_int32), ("heads", ctypes.c_int32), ("k", ctypes.c_int32), ("n", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class AppendParams(ctypes.Structure):
@@ -76,6 +82,7 @@ def _load():
     L.mla_status_string.restype = ctypes.c_char_p
     L.mla_abi_version.argtypes = []
     L.mla_cache_append.argtypes = [ctypes.POINTER(AppendParams), vp, vp, vp, vp, vp, vp, vp, vp]
+    L.mla_head_gemm.argtypes = [ctypes.POINTER(HeadGemmParams), vp, vp, vp, vp]
     for name in EXPORTED:
         if not hasattr(L, name):
             raise ImportError(f"{LIB_PATH} lacks {name}: rebuild it")
@@ -260,4 +267,12 @@ def mla_cache_append(p: AppendParams, c_new, k_rope_new, kv_cache, k_rope_cache,
                               _stream(stream))
     if check:
         _check(st, "mla_cache_append")
+    return st
+
+
+def mla_head_gemm(p: HeadGemmParams, x, w, y, stream=None, check=True) -> int:
+    """Raw C-ABI call of the per-head GEMM y[m, h] = x[m, h] . w[h] (device tensors or addresses)."""
+    st = lib.mla_head_gemm(ctypes.byref(p), _addr(x), _addr(w), _addr(y), _stream(stream))
+    if check:
+        _check(st, "mla_head_gemm")
     return st

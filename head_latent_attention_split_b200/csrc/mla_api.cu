@@ -409,6 +409,28 @@ mla_status_t mla_cache_append(const mla_append_params_t* p, const void* c_new, c
   return mla::launch_cache_append(a, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+mla_status_t mla_head_gemm(const mla_head_gemm_params_t* p, const void* x, const void* w, void* y, void* stream) {
+  if (!p || p->rows < 0 || p->heads < 1 || p->k < 64 || p->n < 64 || p->k % 64 != 0 || p->n % 64 != 0 ||
+      p->reserved != 0)
+    return MLA_ERR_INVALID_ARG;
+  if (p->heads > 65535 || (p->rows + 127) / 128 > 65535) return MLA_ERR_UNSUPPORTED;
+  if (p->rows == 0) return MLA_OK;
+  if (!x || !w || !y) return MLA_ERR_INVALID_ARG;
+  if (((uintptr_t)x | (uintptr_t)w | (uintptr_t)y) & 15) return MLA_ERR_ALIGNMENT;
+  int* status = status_word(current_device());
+  if (!status) return MLA_ERR_CUDA;
+  mla::GemmArgs a{};
+  a.rows = p->rows;
+  a.heads = p->heads;
+  a.k = p->k;
+  a.n = p->n;
+  a.x = x;
+  a.w = w;
+  a.y = y;
+  a.status = status;
+  return mla::launch_head_gemm(a, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 mla_status_t mla_get_device_status(void* stream, int32_t* device_status) {
   if (!device_status) return MLA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MLA_ERR_CUDA;

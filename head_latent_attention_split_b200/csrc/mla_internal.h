@@ -87,4 +87,14 @@ struct AppendArgs {
 };
 cudaError_t launch_cache_append(const AppendArgs& a, cudaStream_t s);
 
+// Arguments of the per-head GEMM (mla_gemm.cu): y[m, h, :] = x[m, h, :] . w[h].
+struct GemmArgs {
+  int rows, heads, k, n;   // k, n multiples of 64
+  const void* x;           // [rows, heads, k] bf16
+  const void* w;           // [heads, k, n] bf16
+  void* y;                 // [rows, heads, n] bf16
+  int* status;
+};
+cudaError_t launch_head_gemm(const GemmArgs& a, cudaStream_t s);
+
 }  // namespace mla

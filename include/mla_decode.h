@@ -252,6 +252,30 @@ mla_status_t mla_cache_append(const mla_append_params_t* params, const void* c_n
                               void* kv_cache, void* k_rope_cache, float* kv_scale, const int32_t* block_table,
                               const int32_t* seq_lens, void* stream);
 
+/* ------------------------------------------------------------------ per-head GEMM
+ *
+ * y[m, h, :] = x[m, h, :] . w[h] for m < rows and every head h: bf16 operands, fp32
+ * accumulation, bf16 result (round to nearest even). The two weight products around the
+ * absorbed decode are instances ("TransMLA: Multi-Head Latent Attention Is All You Need",
+ * sec. 3.4.5, the full MLA structure after conversion: W^UK is absorbed into the query and
+ * W^UV applied to the attention output):
+ *   query absorption     x = q_nope [rows, H, d_h], w[h] = W^UK_h (d_h x r)    -> y = q_lat [rows, H, r]
+ *   output up-projection x = out    [rows, H, r],   w[h] = W^UV_h^T (r x d_v)  -> y [rows, H, d_v]
+ * with rows = B * Sq. Layouts: x [rows][heads][k], w [heads][k][n], y [rows][heads][n],
+ * contiguous device arrays, 16-byte aligned; k and n multiples of 64. Tensor cores (tcgen05,
+ * M = 128 rows per tile, K = 64 per staged chunk). Asynchronous on `stream`, allocates
+ * nothing. Argument errors return at once; a wait timeout sets the sticky status word. */
+typedef struct {
+  int32_t rows;      /* m extent (B * Sq) */
+  int32_t heads;     /* H */
+  int32_t k;         /* contraction length per head */
+  int32_t n;         /* output width per head */
+  int32_t reserved;  /* must be 0 */
+} mla_head_gemm_params_t;
+
+mla_status_t mla_head_gemm(const mla_head_gemm_params_t* params, const void* x, const void* w, void* y,
+                           void* stream);
+
 /* MLA_DECODE_ABI_VERSION of the loaded library. */
 int32_t mla_abi_version(void);
 

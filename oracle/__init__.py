@@ -83,6 +83,9 @@ def lib():
         L.mla_oracle_e4m3_encode_n.restype = None
         L.mla_oracle_cache_append.argtypes = [ctypes.c_int] * 10 + [ctypes.c_double] + [ctypes.c_void_p] * 7
         L.mla_oracle_cache_append.restype = ctypes.c_int
+        L.mla_oracle_head_gemm.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                                                 ctypes.c_void_p]
+        L.mla_oracle_head_gemm.restype = None
         _lib = L
     return _lib
 
@@ -251,3 +254,28 @@ def cache_append(*, B, Sq, r, d_r, block_size, num_blocks, max_blocks_per_seq, i
         B, Sq, r, d_r, block_size, num_blocks, max_blocks_per_seq, in_dtype, cache_dtype, int(bool(rope)),
         float(rope_base), c_new.ctypes.data, k_new.ctypes.data, kv_cache.ctypes.data, ptr(k_rope_cache),
         ptr(kv_scale), bt.ctypes.data, sl.ctypes.data)
+
+
+def _dtype_of(a):
+    if a.dtype == np.float64:
+        return F64
+    if a.dtype == np.float32:
+        return F32
+    if a.dtype == np.uint16:
+        return BF16
+    raise TypeError(a.dtype)
+
+
+def head_gemm(x, w) -> np.ndarray:
+    """y[m, h, :] = x[m, h, :] . w[h] in fp64. x [..., H, k], w [H, k, n]: float32 / float64
+    arrays or bf16 bit patterns (uint16). Returns float64 [..., H, n]."""
+    x = np.ascontiguousarray(x)
+    w = np.ascontiguousarray(w)
+    H, k = x.shape[-2], x.shape[-1]
+    n = w.shape[-1]
+    assert w.shape == (H, k, n), (w.shape, (H, k, n))
+    rows = x.size // (H * k)
+    y = np.empty((*x.shape[:-2], H, n), dtype=np.float64)
+    lib().mla_oracle_head_gemm(rows, H, k, n, _dtype_of(x), x.ctypes.data, _dtype_of(w), w.ctypes.data,
+                               y.ctypes.data)
+    return y

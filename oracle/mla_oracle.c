@@ -421,3 +421,23 @@ int mla_oracle_cache_append(int B, int Sq, int r, int d_r, int bs, int num_block
   }
   return err;
 }
+
+/* ------------------------------------------------------------------ per-head products
+ *
+ * y[m, h, j] = sum_k x[m, h, k] * w[h, k, j] in fp64 from bf16 / f32 / f64 storage: the query
+ * absorption (w[h] = W^UK_h) and the output up-projection (w[h] = W^UV_h^T) around the
+ * absorbed decode ("TransMLA: Multi-Head Latent Attention Is All You Need", sec. 3.4.5).
+ */
+void mla_oracle_head_gemm(int rows, int heads, int k, int n, int x_dtype, const void* x, int w_dtype, const void* w,
+                          double* y) {
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int m = 0; m < rows; ++m)
+    for (int h = 0; h < heads; ++h) {
+      double* yr = y + ((size_t)m * heads + h) * n;
+      for (int j = 0; j < n; ++j) yr[j] = 0.0;
+      for (int kk = 0; kk < k; ++kk) {
+        const double xv = load_elem(x, x_dtype, ((size_t)m * heads + h) * k + kk);
+        for (int j = 0; j < n; ++j) yr[j] += xv * load_elem(w, w_dtype, ((size_t)h * k + kk) * n + j);
+      }
+    }
+}
