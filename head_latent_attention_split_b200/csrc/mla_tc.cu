@@ -15,21 +15,22 @@
 //    stage, 4 stages). The query's RoPE part stays in shared memory (8 KB).
 //  * QK: S_j[128 x 64] = Q_j . C_j^T over the CTA's 288 channels (16 MMAs with A in
 //    TMEM + 2 with A in shared memory, K = 16 each). The full score is S_0 + S_1.
-//  * Row split of the softmax: CTA j normalises the 64 rows in TMEM lane quarters
-//    2 j and 2 j + 1 ("own" rows); the other 64 are the peer's. Per tile:
-//      - the 4 warps on the peer's quarters read those rows of S_j and store them with
-//        st.async straight into the peer's receive buffer (16 KB; bytes complete on
-//        the peer's mbarrier);
-//      - the 4 warps on the own quarters add the peer's partials to their own, take
-//        the row maximum (two warps per row, 32 columns each), the exponentials and
-//        the row sums, write P into TMEM and st.async the same bf16 rows (8 KB) plus
-//        one rescale factor per row to the peer;
-//      - the peer-quarter warps then write the received P rows into their TMEM and,
-//        when the owner moved a row's running maximum, rescale those O rows.
-//    Only 24.25 KB cross the pair per tile and direction, every exponential is taken
-//    once, and the exchange of a tile overlaps the exponentials of the previous one.
-//    The running maximum only moves when a tile raises it by more than 2^8, so O is
-//    rescaled rarely.
+//  * Row split of the softmax: in every TMEM lane quarter q, lanes [32 q + 16 j, +16)
+//    hold CTA j's own rows and the other 16 lanes the peer's, read and written with the
+//    16-lane TMEM shape. Warp q (0-3) works on the own lanes of quarter q, warp q + 4 on
+//    the peer lanes, so both kinds of work spread over the four SM sub-partitions, and a
+//    row's 64 columns live in one warp (threads t and t + 16). Per tile:
+//      - the peer-lane warps stage those rows of S_j (fp32) and move each quarter to the
+//        peer with one bulk copy (bytes complete on the peer's mbarrier);
+//      - the own-lane warps add the peer's partials to theirs, take the row maximum (a
+//        shuffle), the exponentials (each once, in the row's owner) and the row sums,
+//        write P into TMEM and send the same bf16 rows plus one rescale factor per row
+//        back the same way;
+//      - the peer-lane warps write the received P rows into their TMEM lanes and
+//        rescale those O rows when the owner moved a maximum. They serve their two
+//        streams (ship scores, take probabilities) as an event loop.
+//    24.25 KB cross the pair per tile and direction. The running maximum only moves
+//    when a tile raises it by more than 2^8, so O is rescaled rarely.
 //  * PV: O_j[128 x 256] += P[128 x 64] . C_j[64 x 256] with A = P from TMEM and B =
 //    the SAME shared-memory tile the QK used, read N-major (4 MMAs, N = 256). The MMA
 //    issuer runs QK(k) then PV(k - 2).
@@ -42,10 +43,10 @@
 //    (2^-16 relative). The score MMAs then give S_t / s_t; the softmax multiplies each
 //    column by s_t, and P by s_t before PV (sum_t p_t s_t code_t = sum_t p_t c_t), with
 //    the row sum over the unscaled p_t.
-//  * Warp roles: warps 0-7 softmax / exchange / epilogue, warp 8 TMA producer, warp 9
-//    TMEM allocator and single-thread MMA issuer, warps 10-11 FP8 converters; mbarrier
-//    pipelines between them. Every wait is bounded (timeout -> MLA_ERR_TIMEOUT, clean
-//    exit).
+//  * Warp roles: warps 0-3 own-lane softmax and epilogue, warps 4-7 peer-lane exchange
+//    and epilogue, warp 8 TMA producer, warp 9 TMEM allocator and single-thread MMA
+//    issuer, warps 10-11 FP8 converters; mbarrier pipelines between them. Every wait is
+//    bounded (timeout -> MLA_ERR_TIMEOUT, clean exit).
 // The work split over workers (CTA pairs) is the flat block list plan of mla_device.cuh.
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -97,6 +98,7 @@ template <bool kFp8> struct Geo {
   static constexpr uint32_t kSmemBytes = kOffCtl + kCtlBytes + 1024;   // + alignment slack
 };
 static_assert(Geo<true>::kOffScale + 256 <= Geo<true>::kStageBytes && Geo<true>::kStageBytes % 1024 == 0, "fp8 stage");
+static_assert(Geo<false>::kOffScale == Geo<true>::kOffScale, "one stage geometry for both caches");
 static_assert(Geo<false>::kOffQr % 1024 == 0 && Geo<true>::kOffQr % 1024 == 0, "buffers need 1024-byte alignment");
 static_assert(Geo<false>::kSmemBytes <= 232448 && Geo<true>::kSmemBytes <= 232448, "shared memory budget");
 static_assert(kRxPBytes % 16 == 0 && Geo<true>::kOffTxS % 16 == 0 && Geo<false>::kOffTxS % 16 == 0,
@@ -134,15 +136,11 @@ struct Ctl {
   uint64_t rxp_full;        // the peer's probabilities and rescale factors of the next tile landed
   uint64_t txs_ok[2];       // the peer has read the partial scores we last sent into its buffer b
   uint64_t txp_ok;          // ... the probabilities
-  uint64_t mx[2];           // the two warps sharing 32 own rows published their tile maxima
-  uint64_t lx[2];           // ... their row sums
   uint64_t lrx_full[2];     // the peer's row sums of segment s, s & 1 == b, have landed
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
   WorkerPlan plan;
-  float mbuf[2][2][64];     // [tile parity][half][own row]
-  float lbuf[2][64];        // [half][own row]
   float lrx[2][64];         // [segment parity][peer's own row]: written by the peer
 };
 static_assert(sizeof(Ctl) <= kCtlBytes, "control block too large");
@@ -199,8 +197,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
       mbar_init(smem_u32(&ctl.lrx_full[i]), 1);
       mbar_arrive_expect_tx(smem_u32(&ctl.lrx_full[i]), kLrxBytes);
       mbar_init(smem_u32(&ctl.txs_ok[i]), 4);   // one arrival per consuming warp of the peer
-      mbar_init(smem_u32(&ctl.mx[i]), 64);
-      mbar_init(smem_u32(&ctl.lx[i]), 64);
     }
     for (int i = 0; i < kStages; ++i) {
       mbar_init(smem_u32(&ctl.kv_ready[i]), kConvThreads);
