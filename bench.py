@@ -95,6 +95,23 @@ def measured_traffic(wl, model, kernel):
     return None if per_tok is None else per_tok * model["tokens"]
 
 
+def reduce_max(x: float, world: int, device=None) -> float:
+    """Max of x over the ranks of the default process group (x itself when world == 1)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate_tbs(world: int, steps: int, bytes_per_step: float, max_ms: float) -> float:
+    """Whole-job rate in TB/s: each of `world` replicas moves bytes_per_step per step, and the job
+    lasts as long as its slowest rank (max_ms for `steps` steps)."""
+    return world * steps * bytes_per_step / (max_ms / 1e3) / 1e12
+
+
 def work_model(inp):
     """Algorithmic bytes and FLOPs of one step ('Algorithmic work')."""
     w = inp["workload"]
@@ -407,11 +424,7 @@ def main():
     step_ms = [e[0].elapsed_time(e[2]) for e in evs]
     dec_ms = [e[0].elapsed_time(e[1]) for e in evs]
     comb_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    total_ms = sum(step_ms)
-    tot = torch.tensor([total_ms], dtype=torch.float64, device=out.device)
-    if world > 1:
-        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
-    total_ms = float(tot.item())
+    total_ms = reduce_max(sum(step_ms), world, out.device)
     st = mla.device_status()
     if st != 0:
         raise RuntimeError(f"device status {mla.status_string(st)}")
@@ -438,10 +451,7 @@ def main():
         b.synchronize()
         if i >= 2:
             e2e_ms += a.elapsed_time(b)
-    e2e = torch.tensor([e2e_ms], dtype=torch.float64, device=out.device)
-    if world > 1:
-        dist.all_reduce(e2e, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e.item())
+    e2e_ms = reduce_max(e2e_ms, world, out.device)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -450,7 +460,7 @@ def main():
     if rank == 0:
         peaks = load_peaks()
         sec = total_ms / 1e3
-        value = world * K * model["cache_bytes"] / sec / 1e12
+        value = job_rate_tbs(world, K, model["cache_bytes"], total_ms)
         dec_s = statistics.mean(dec_ms) / 1e3
         t_hbm = model["bytes"] / (peaks["hbm_gbs"] * 1e9)
         t_tc = model["flops"] / (peaks["bf16_tflops"] * 1e12)
@@ -485,7 +495,7 @@ def main():
                 roofline_us=1e6 * max(t_hbm, t_tc), step_frac=max(t_hbm, t_tc) / (total_ms / K / 1e3),
                 peaks=peaks),
             cpu_baseline=cpu,
-            e2e=dict(value=world * E * model["cache_bytes"] / (e2e_ms / 1e3) / 1e12, unit="TB/s",
+            e2e=dict(value=job_rate_tbs(world, E, model["cache_bytes"], e2e_ms), unit="TB/s",
                      h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms / E) if E > 0 else None,
             gpu_launches=2 * K,
             clocks=clocks,
