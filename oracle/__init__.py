@@ -86,6 +86,11 @@ def lib():
         L.mla_oracle_head_gemm.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
                                                                  ctypes.c_void_p]
         L.mla_oracle_head_gemm.restype = None
+        L.mla_oracle_dsa_index.argtypes = [ctypes.c_int] * 9 + [ctypes.c_void_p] * 8 + [ctypes.c_int]
+        L.mla_oracle_dsa_index.restype = ctypes.c_int
+        L.mla_oracle_decode_sparse.argtypes = [P, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, dp, dp,
+                                               ctypes.c_int]
+        L.mla_oracle_decode_sparse.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -279,3 +284,94 @@ def head_gemm(x, w) -> np.ndarray:
     lib().mla_oracle_head_gemm(rows, H, k, n, _dtype_of(x), x.ctypes.data, _dtype_of(w), w.ctypes.data,
                                y.ctypes.data)
     return y
+
+
+# ---------------------------------------------------------------------------------------
+# DeepSeek Sparse Attention: "TransMLA & Sparse Latent Attention" lesson, Chapter 6 ("The
+# lightning indexer", "Fine-grained token selection") and Chapter 7 ("DSA runs in MLA's
+# MQA mode"). Parity status: pinned by tests/test_dsa_pins.py.
+
+def attended_counts(seq_lens, Sq, causal) -> np.ndarray:
+    """Tokens each query row (b, s) may see: [B, Sq] int64 (the decode's causal rule)."""
+    L = np.asarray(seq_lens, dtype=np.int64)[:, None]
+    s = np.arange(Sq, dtype=np.int64)[None, :]
+    n = L - Sq + 1 + s if causal else np.broadcast_to(L, (L.shape[0], Sq))
+    return np.maximum(n, 0)
+
+
+def dsa_index(q_codes, q_scale, weights, k_codes, k_scale, block_table, seq_lens, *, causal=False,
+              max_seq_len=None, block_size=64, nthreads=0) -> np.ndarray:
+    """Lightning-indexer scores in fp64 (see mla_oracle.c).
+
+    q_codes uint8 e4m3 [B, Sq, HI, dI], q_scale / weights float32 [B, Sq, HI], k_codes
+    uint8 e4m3 [num_blocks, bs, dI], k_scale float32 [num_blocks, bs]. Returns float64
+    [B, Sq, max_seq_len]; entries past a row's attended count are NaN.
+    """
+    q_codes = np.ascontiguousarray(q_codes, dtype=np.uint8)
+    q_scale = np.ascontiguousarray(q_scale, dtype=np.float32)
+    weights = np.ascontiguousarray(weights, dtype=np.float32)
+    k_codes = np.ascontiguousarray(k_codes, dtype=np.uint8)
+    k_scale = np.ascontiguousarray(k_scale, dtype=np.float32)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    B, Sq, HI, dI = q_codes.shape
+    num_blocks = k_codes.shape[0]
+    if max_seq_len is None:
+        max_seq_len = int(sl.max()) if sl.size else 0
+    out = np.full((B, Sq, max_seq_len), np.nan, dtype=np.float64)
+    _check(lib().mla_oracle_dsa_index(B, Sq, HI, dI, block_size, num_blocks, bt.shape[1], int(bool(causal)),
+                                      max_seq_len, q_codes.ctypes.data, q_scale.ctypes.data,
+                                      weights.ctypes.data, k_codes.ctypes.data, k_scale.ctypes.data,
+                                      bt.ctypes.data, sl.ctypes.data, out.ctypes.data, nthreads))
+    return out
+
+
+def dsa_counts(n_rows, k: int) -> np.ndarray:
+    """Tokens a query row keeps: all of its n candidates while n <= k, else k
+    (Chapter 6, "Worked arithmetic": min(t, k) per query)."""
+    return np.minimum(np.maximum(np.asarray(n_rows, dtype=np.int64), 0), k)
+
+
+def dsa_topk(scores, n_rows, k: int):
+    """Top-k selection ("Fine-grained token selection"): for each row, the positions of
+    the k highest of its first n scores (all n when n <= k). Equal scores are taken
+    lowest position first, so the set is unique. Returns (indices int32 [..., k] in
+    ascending position order, -1 past the count; counts int32 [...]).
+    A stable sort of (-score, position) is the selection step."""
+    scores = np.asarray(scores)
+    n_rows = np.asarray(n_rows, dtype=np.int64)
+    lead = scores.shape[:-1]
+    assert n_rows.shape == lead, (n_rows.shape, lead)
+    flat = scores.reshape(-1, scores.shape[-1])
+    nf = n_rows.reshape(-1)
+    idx = np.full((flat.shape[0], k), -1, dtype=np.int32)
+    cnt = dsa_counts(nf, k).astype(np.int32)
+    for i in range(flat.shape[0]):
+        n = int(nf[i])
+        if n <= 0:
+            continue
+        pos = np.arange(n)
+        if n > k:
+            order = np.lexsort((pos, -flat[i, :n]))   # score descending, then position
+            pos = np.sort(order[:k])
+        idx[i, :len(pos)] = pos
+    return idx.reshape(lead + (k,)), cnt.reshape(lead)
+
+
+def decode_sparse(q_lat, q_rope, kv_cache, block_table, seq_lens, softmax_scale, indices, counts,
+                  k_rope_cache=None, kv_scale=None, block_size=64, nthreads=0):
+    """MLA decode of each query row over its selected tokens only, fp64.
+
+    indices int32 [B, Sq, top_k] (positions of sequence b), counts int32 [B, Sq]. Returns
+    (out [B, Sq, H, r] f64, lse [B, Sq, H] f64)."""
+    bd = _Bound(q_lat, q_rope, kv_cache, block_table, seq_lens, softmax_scale, False,
+                k_rope_cache, kv_scale, block_size)
+    B, Sq, H, r, _ = bd.shape
+    indices = np.ascontiguousarray(indices, dtype=np.int32)
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    assert indices.shape[:2] == (B, Sq) and counts.shape == (B, Sq)
+    out = np.zeros((B, Sq, H, r), dtype=np.float64)
+    lse = np.zeros((B, Sq, H), dtype=np.float64)
+    _check(lib().mla_oracle_decode_sparse(ctypes.byref(bd.p), indices.shape[2], indices.ctypes.data,
+                                          counts.ctypes.data, _dp(out), _dp(lse), nthreads))
+    return out, lse

@@ -140,17 +140,14 @@ static void gather_tokens(const mla_oracle_problem* p, int b, int64_t t0, int64_
 }
 
 /*
- * One (b, s, h) row over the token window [t0, t1) intersected with what the row may
- * attend to. toks holds the decoded tokens [t0, t1). sigma is scratch of t1 - t0.
+ * Query row qrow (= (b * Sq + s) * H + h) against the n decoded tokens in toks (row k:
+ * c then kR). sigma is scratch of n. n = 0 gives out = 0, lse = -inf.
  */
-static void decode_row(const mla_oracle_problem* p, int b, int s, int h, int64_t t0, int64_t t1,
-                       const double* toks, double* sigma, double* out, double* lse) {
+static void softmax_row(const mla_oracle_problem* p, size_t qrow, int64_t n, const double* toks, double* sigma,
+                        double* out, double* lse) {
   const int D = p->r + p->d_r;
-  int64_t n = attended(p, p->seq_lens[b], s);
-  int64_t hi = t1 < n ? t1 : n;
-  size_t qrow = ((size_t)b * p->Sq + s) * p->H + h;
   for (int k = 0; k < p->r; ++k) out[k] = 0.0;
-  if (hi <= t0) {
+  if (n <= 0) {
     *lse = -INFINITY;
     return;
   }
@@ -161,26 +158,37 @@ static void decode_row(const mla_oracle_problem* p, int b, int s, int h, int64_t
 
   /* pass 1: scores and their maximum */
   double M = -INFINITY;
-  for (int64_t t = t0; t < hi; ++t) {
-    const double* c = toks + (size_t)(t - t0) * D;
+  for (int64_t t = 0; t < n; ++t) {
+    const double* c = toks + (size_t)t * D;
     double content = 0.0, positional = 0.0;
     for (int k = 0; k < p->r; ++k) content += qv[k] * c[k];
     for (int j = 0; j < p->d_r; ++j) positional += qv[p->r + j] * c[p->r + j];
     double sg = p->softmax_scale * (content + positional);
-    sigma[t - t0] = sg;
+    sigma[t] = sg;
     if (sg > M) M = sg;
   }
   /* pass 2: normaliser, log-sum-exp, weighted sum of latents */
   double Z = 0.0;
-  for (int64_t t = t0; t < hi; ++t) Z += exp(sigma[t - t0] - M);
+  for (int64_t t = 0; t < n; ++t) Z += exp(sigma[t] - M);
   double L = M + log(Z);
-  for (int64_t t = t0; t < hi; ++t) {
-    double w = exp(sigma[t - t0] - L);
-    const double* c = toks + (size_t)(t - t0) * D;
+  for (int64_t t = 0; t < n; ++t) {
+    double w = exp(sigma[t] - L);
+    const double* c = toks + (size_t)t * D;
     for (int k = 0; k < p->r; ++k) out[k] += w * c[k];
   }
   *lse = L;
   if (qv != qv_stack) free(qv);
+}
+
+/*
+ * One (b, s, h) row over the token window [t0, t1) intersected with what the row may
+ * attend to. toks holds the decoded tokens [t0, t1). sigma is scratch of t1 - t0.
+ */
+static void decode_row(const mla_oracle_problem* p, int b, int s, int h, int64_t t0, int64_t t1,
+                       const double* toks, double* sigma, double* out, double* lse) {
+  int64_t n = attended(p, p->seq_lens[b], s);
+  int64_t hi = t1 < n ? t1 : n;
+  softmax_row(p, ((size_t)b * p->Sq + s) * p->H + h, hi - t0, toks, sigma, out, lse);
 }
 
 /*
@@ -440,4 +448,136 @@ void mla_oracle_head_gemm(int rows, int heads, int k, int n, int x_dtype, const 
         for (int j = 0; j < n; ++j) yr[j] += xv * load_elem(w, w_dtype, ((size_t)h * k + kk) * n + j);
       }
     }
+}
+
+/*
+ * ---------------------------------------------------------------------------------
+ * DeepSeek Sparse Attention (DSA) over the same paged cache: "TransMLA & Sparse Latent
+ * Attention" lesson, Chapter 6 ("The lightning indexer", "Fine-grained token selection")
+ * and Chapter 7 ("The indexer keeps its own small cache", "DSA runs in MLA's MQA mode").
+ *
+ * Indexer score of cached token t for query row (b, s), H^I indexer heads:
+ *     I_t = sum_j w[b,s,j] * ReLU( q_j . k_t )
+ * q_j = e4m3(q_codes[b,s,j,:]) * q_scale[b,s,j]; k_t = e4m3(k_codes[slot(t),:]) * k_scale[slot(t)].
+ * The pages run the indexer in FP8 and give no scale layout; the reading here is one
+ * fp32 scale per stored vector (per indexer head of a query, per cached token), the
+ * same per-token scheme as the FP8 latent cache. The key side-cache k_codes
+ * [num_blocks, bs, d^I] shares the latent cache's block table. Query row s sees the
+ * first L - Sq + 1 + s tokens when causal, else all L.
+ * scores: [B, Sq, max_seq_len] double; entries past a row's attended count are left
+ * as they are.
+ */
+int mla_oracle_dsa_index(int B, int Sq, int HI, int dI, int bs, int num_blocks, int max_blocks, int causal,
+                         int max_seq_len, const uint8_t* q_codes, const float* q_scale, const float* w,
+                         const uint8_t* k_codes, const float* k_scale, const int32_t* block_table,
+                         const int32_t* seq_lens, double* scores, int nthreads) {
+  if (B < 0 || Sq < 1 || HI < 1 || dI < 1 || dI > 1024 || bs < 1 || num_blocks < 0 || max_blocks < 0 ||
+      max_seq_len < 0)
+    return OR_ERR_ARG;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+  for (int b = 0; b < B; ++b) {
+    const int64_t L = seq_lens[b];
+    if (L < 0 || L > (int64_t)max_blocks * bs || L > max_seq_len) return OR_ERR_SEQ_LEN;
+    for (int64_t i = 0; i < (L + bs - 1) / bs; ++i) {
+      const int32_t blk = block_table[(size_t)b * max_blocks + i];
+      if (blk < 0 || blk >= num_blocks) return OR_ERR_BLOCK_ID;
+    }
+  }
+  double* q = (double*)malloc(sizeof(double) * (size_t)HI * dI);
+  if (!q) return OR_ERR_NOMEM;
+  for (int b = 0; b < B; ++b) {
+    const int64_t L = seq_lens[b];
+    for (int s = 0; s < Sq; ++s) {
+      int64_t n = causal ? L - Sq + 1 + s : L;
+      if (n < 0) n = 0;
+      const size_t qrow = (size_t)b * Sq + s;
+      for (int j = 0; j < HI; ++j) {
+        const double qs = (double)q_scale[qrow * HI + j];
+        for (int d = 0; d < dI; ++d)
+          q[(size_t)j * dI + d] = mla_oracle_e4m3_to_double(q_codes[(qrow * HI + j) * dI + d]) * qs;
+      }
+      double* out = scores + qrow * (size_t)max_seq_len;
+#pragma omp parallel for schedule(static)
+      for (int64_t t = 0; t < n; ++t) {
+        const int32_t blk = block_table[(size_t)b * max_blocks + t / bs];
+        const size_t slot = (size_t)blk * bs + (size_t)(t % bs);
+        const double ks = (double)k_scale[slot];
+        double kt[1024];
+        for (int d = 0; d < dI; ++d) kt[d] = mla_oracle_e4m3_to_double(k_codes[slot * dI + d]) * ks;
+        double I = 0.0;
+        for (int j = 0; j < HI; ++j) {
+          double dot = 0.0;
+          for (int d = 0; d < dI; ++d) dot += q[(size_t)j * dI + d] * kt[d];
+          I += (double)w[qrow * HI + j] * (dot > 0.0 ? dot : 0.0);
+        }
+        out[t] = I;
+      }
+    }
+  }
+  free(q);
+  return OR_OK;
+}
+
+/*
+ * MLA decode over selected tokens (Chapter 7, "DSA runs in MLA's MQA mode": the
+ * selected cache entries are attended in the absorbed form, one latent shared by every
+ * head). Query row (b, s) attends exactly the tokens indices[b, s, 0 .. counts[b, s])
+ * of sequence b (positions, mapped through the block table); same score, softmax and
+ * value as the dense decode above. indices: [B, Sq, top_k], counts: [B, Sq].
+ */
+int mla_oracle_decode_sparse(const mla_oracle_problem* p, int top_k, const int32_t* indices,
+                             const int32_t* counts, double* out, double* lse, int nthreads) {
+  int rc = check_problem(p);
+  if (rc) return rc;
+  if (top_k < 0) return OR_ERR_ARG;
+  const int D = p->r + p->d_r;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+  /* the list's tokens, decoded, as a window [0, n) of a one-row-per-token buffer */
+  double* toks = (double*)malloc(sizeof(double) * (size_t)(top_k > 0 ? top_k : 1) * D);
+  if (!toks) return OR_ERR_NOMEM;
+  int err = OR_OK;
+  for (int b = 0; b < p->B && !err; ++b) {
+    for (int s = 0; s < p->Sq && !err; ++s) {
+      const size_t row = (size_t)b * p->Sq + s;
+      const int n = counts[row];
+      if (n < 0 || n > top_k) {
+        err = OR_ERR_ARG;
+        break;
+      }
+      for (int i = 0; i < n; ++i) {
+        const int32_t t = indices[row * top_k + i];
+        if (t < 0 || t >= p->seq_lens[b]) {
+          err = OR_ERR_ARG;
+          break;
+        }
+        gather_tokens(p, b, t, t + 1, toks + (size_t)i * D);
+      }
+      if (err) break;
+#pragma omp parallel
+      {
+        double* sigma = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+        if (!sigma) {
+#pragma omp atomic write
+          err = OR_ERR_NOMEM;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+          for (int h = 0; h < p->H; ++h) {
+            const size_t o = row * p->H + h;
+            softmax_row(p, o, n, toks, sigma, out + o * p->r, lse + o);
+          }
+          free(sigma);
+        }
+      }
+    }
+  }
+  free(toks);
+  return err;
 }

@@ -280,3 +280,73 @@ def to_torch(inp: dict, device="cuda") -> dict:
                                    "seq_lens")}
     out["workload"] = inp["workload"]
     return out
+
+
+# ---------------------------------------------------------------------------------------
+# DeepSeek Sparse Attention inputs ("TransMLA & Sparse Latent Attention" lesson, Chapter 6
+# "The lightning indexer": H^I = 64 indexer heads of width d^I = 128, top k = 2048 of a
+# 128K context). The indexer's query and its key side-cache are stored as e4m3 codes with
+# one fp32 scale per vector (per indexer head of a query row; per cached token), the
+# per-head weights as fp32. The key side-cache shares the latent cache's block table.
+
+@dataclass(frozen=True)
+class DsaWorkload:
+    """A sparse decode problem: the latent-cache decode workload plus the indexer's shapes."""
+    name: str
+    mla: Workload
+    HI: int = 64
+    dI: int = 128
+    top_k: int = 2048
+    w_std: float = 1.0 / 8.0
+    description: str = ""
+
+    @property
+    def seed(self) -> int:
+        return self.mla.seed
+
+
+DSA_WORKLOADS = [
+    DsaWorkload(
+        "dsa_small",
+        Workload(name="dsa_small_mla", B=3, Sq=1, H=32, r=512, d_r=64, seq_lens=(300, 4100, 2500),
+                 q_std=1.0, c_std=1.0 / math.sqrt(512.0), outlier_frac=0.01, seed=1100),
+        top_k=512,
+        description="small sparse decode: B=3 H=32, L = 300 / 4100 / 2500 (one list shorter than k), k=512"),
+    DsaWorkload(
+        "dsa_v32",
+        Workload(name="dsa_v32_mla", B=32, Sq=1, H=128, r=512, d_r=64, seq_lens=(131072,) * 32,
+                 q_std=1.0, c_std=1.0 / math.sqrt(512.0), outlier_frac=0.01, seed=1101),
+        description="DeepSeek-V3.2-shaped sparse decode: B=32 H=128 at the end of a 128K context, "
+                    "indexer 64 heads x 128 (FP8), top 2048"),
+]
+DSA_BY_NAME = {w.name: w for w in DSA_WORKLOADS}
+
+
+def make_dsa_inputs(w: DsaWorkload, threads: int | None = None, with_cache: bool = True) -> dict:
+    """Inputs of one sparse decode step: the latent-cache decode inputs of ``w.mla`` (unless
+    ``with_cache`` is False) plus the indexer query codes / scales / weights and the key
+    side-cache (host numpy)."""
+    threads = threads or min(16, os.cpu_count() or 1)
+    res = make_inputs(w.mla, threads) if with_cache else None
+    m = w.mla
+    lens = resolve_seq_lens(m)
+    bs = m.block_size
+    if res is None:
+        # the same block table as make_inputs (identical draws), without the latent cache
+        tmp = make_inputs(m.with_(r=2, d_r=0, cache_dtype=F32, q_dtype=F32), threads)
+        block_table, num_blocks = tmp["block_table"], tmp["num_blocks"]
+        res = dict(workload=m, seq_lens=lens, block_table=block_table, num_blocks=num_blocks,
+                   max_blocks_per_seq=block_table.shape[1])
+    num_blocks = res["num_blocks"]
+    ss_q, ss_w, ss_k = np.random.SeedSequence([m.seed, 23]).spawn(3)
+    q = _fill_normal(ss_q, m.B * m.Sq * w.HI * w.dI, threads).reshape(m.B, m.Sq, w.HI, w.dI)
+    wts = _fill_normal(ss_w, m.B * m.Sq * w.HI, threads).reshape(m.B, m.Sq, w.HI) * np.float32(w.w_std)
+    k = _fill_normal(ss_k, num_blocks * bs * w.dI, threads).reshape(num_blocks, bs, w.dI)
+    q_codes, q_scale = quantize_e4m3_per_token(q)
+    k_codes, k_scale = quantize_e4m3_per_token(k)
+    if "poison" in res:   # slots no sequence may read hold NaN here too
+        k_codes[res["poison"]] = E4M3_NAN
+        k_scale[res["poison"]] = np.nan
+    res.update(dsa=w, iq_codes=q_codes, iq_scale=q_scale, iw=wts.astype(np.float32), ik_codes=k_codes,
+               ik_scale=k_scale, top_k=w.top_k, max_seq_len=int(lens.max()) if lens.size else 0)
+    return res
