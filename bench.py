@@ -51,9 +51,11 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--op", default="decode", choices=["decode", "append", "absorb", "project"],
+    ap.add_argument("--op", default="decode", choices=["decode", "append", "absorb", "project", "dsa"],
                     help="decode: the decode step (default); append: the paged cache append of the step's new "
-                         "tokens; absorb / project: the per-head W^UK / W^UV products around the decode")
+                         "tokens; absorb / project: the per-head W^UK / W^UV products around the decode; dsa: "
+                         "the sparse decode step (indexer, top-k, decode over the selected tokens)")
+    ap.add_argument("--dsa-workload", default="dsa_v32", choices=list(W.DSA_BY_NAME))
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller profiling captures only)")
     return ap.parse_args()
@@ -338,6 +340,150 @@ def head_gemm_arm(args, rank, local):
             gpu_launches=args.steps)), flush=True)
 
 
+def dsa_work_model(inp):
+    """Algorithmic bytes / FLOPs of one sparse decode step, per kernel."""
+    dw = inp["dsa"]
+    w = inp["workload"]
+    n = np.asarray(inp["seq_lens"], np.int64)            # q_len 1: each row sees its whole sequence
+    cnt = np.minimum(n, dw.top_k)
+    rows = w.B * w.Sq
+    idx_bytes = int(n.sum()) * (dw.dI + 4 + 4) + rows * dw.HI * (dw.dI + 8)     # key codes + scale, score out; query
+    idx_flops = int(n.sum()) * dw.HI * dw.dI * 2
+    topk_bytes = int(n.sum()) * 4 + rows * dw.top_k * 4                         # scores in, positions out
+    dec_bytes = int(cnt.sum()) * (w.r + w.d_r) * 2 + rows * w.H * ((w.r + w.d_r) * 2 + w.r * 2 + 4)
+    dec_flops = int(cnt.sum()) * w.H * (2 * (w.r + w.d_r) + 2 * w.r)
+    return dict(index=dict(bytes=idx_bytes, flops=idx_flops), topk=dict(bytes=topk_bytes, flops=0),
+                decode=dict(bytes=dec_bytes, flops=dec_flops), tokens=int(n.sum()), selected=int(cnt.sum()))
+
+
+def dsa_cpu_baseline(inp, seconds):
+    """The oracle's three steps on whole query rows until `seconds` elapse."""
+    import oracle
+    w = inp["workload"]
+    cores = os.cpu_count() or 1
+    elapsed, nrow, b = 0.0, 0, 0
+    while elapsed < seconds and nrow < w.B:
+        sl = slice(b, b + 1)
+        L = int(inp["seq_lens"][b])
+        t0 = time.perf_counter()
+        sc = oracle.dsa_index(inp["iq_codes"][sl], inp["iq_scale"][sl], inp["iw"][sl], inp["ik_codes"],
+                              inp["ik_scale"], inp["block_table"][sl], inp["seq_lens"][sl], max_seq_len=L,
+                              nthreads=cores)
+        idx, cnt = oracle.dsa_topk(sc, np.array([[L]]), inp["top_k"])
+        oracle.decode_sparse(inp["q_lat"][sl], inp["q_rope"][sl], inp["kv_cache"], inp["block_table"][sl],
+                             inp["seq_lens"][sl], w.scale, idx, cnt, nthreads=cores)
+        elapsed += time.perf_counter() - t0
+        nrow += 1
+        b += 1
+    return dict(value=nrow / w.B / elapsed, unit="steps/s", cores=cores, kind="oracle",
+                sample=f"{nrow} of {w.B} sequences (indexer over the full context, top-k, sparse decode of all "
+                       f"{w.H} heads), {elapsed:.1f} s of fp64 CPU work")
+
+
+def dsa_arm(args, rank, local):
+    """Time one sparse decode step: mla_dsa_index + mla_dsa_topk + mla_sparse_decode."""
+    import torch
+    import head_latent_attention_split_b200 as mla
+    dw = W.DSA_BY_NAME[args.dsa_workload]
+    if args.batch:
+        m = dw.mla
+        dw = W.DsaWorkload(f"{dw.name}_b{args.batch}", m.with_(B=args.batch, seq_lens=tuple(m.seq_lens[:1]) * args.batch),
+                           dw.HI, dw.dI, dw.top_k, dw.w_std)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    inp = W.make_dsa_inputs(dw)
+    w = inp["workload"]
+    t = W.to_torch(inp, dev)
+    g = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).to(dev) for k in ("iq_codes", "iq_scale", "iw", "ik_codes",
+                                                                              "ik_scale")}
+    L, k = inp["max_seq_len"], dw.top_k
+    scores = torch.empty((w.B, 1, L), dtype=torch.float32, device=dev)
+    idx = torch.empty((w.B, 1, k), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, 1), dtype=torch.int32, device=dev)
+    dp = mla.dsa_params_for(g["iq_codes"], g["ik_codes"], t["block_table"], L, k)
+    p = mla.params_for(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], w.scale, False, kernel="tcgen05")
+    ws = torch.empty(max(1, mla.workspace_size(p)), dtype=torch.uint8, device=dev)
+    out = torch.empty(t["q_lat"].shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(t["q_lat"].shape[:3], dtype=torch.float32, device=dev)
+
+    def step(ev):
+        ev[0].record()
+        mla.mla_dsa_index(dp, g["iq_codes"], g["iq_scale"], g["iw"], g["ik_codes"], g["ik_scale"], t["block_table"],
+                          t["seq_lens"], scores)
+        ev[1].record()
+        mla.mla_dsa_topk(dp, scores, t["seq_lens"], idx, cnt)
+        ev[2].record()
+        mla.mla_sparse_decode(p, k, t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], idx, cnt, out, lse, ws)
+        ev[3].record()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K + max(3, args.warmup))]
+    for e in evs:
+        for x in e:
+            x.record()
+    for i in range(max(3, args.warmup)):
+        step(evs[K + i])
+    torch.cuda.synchronize()
+    st = mla.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {mla.status_string(st)}")
+    props = torch.cuda.get_device_properties(local)
+    gpu_id = getattr(props, "uuid", None)
+    sampler = ClockSampler(f"GPU-{gpu_id}" if gpu_id is not None else local)
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    sampler.mark_start()
+    for i in range(K):
+        step(evs[i])
+    torch.cuda.synchronize()
+    sampler.mark_end()
+    clocks = sampler.stop()
+    st = mla.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {mla.status_string(st)}")
+    ms = {name: [e[i].elapsed_time(e[i + 1]) for e in evs[:K]] for i, name in enumerate(("index", "topk", "decode"))}
+    total_ms = sum(evs[i][0].elapsed_time(evs[i][3]) for i in range(K))
+    model = dsa_work_model(inp)
+    peaks = load_peaks()
+    detail = {}
+    for name in ("index", "topk", "decode"):
+        sec = statistics.mean(ms[name]) / 1e3
+        d = model[name]
+        t_hbm, t_tc = d["bytes"] / (peaks["hbm_gbs"] * 1e9), d["flops"] / (peaks["bf16_tflops"] * 1e12)
+        if name == "index":
+            t_tc /= 2.0    # e4m3 MMA: twice the bf16 dense rate (nominal ratio)
+        detail[name] = dict(ms=1e3 * sec, algorithmic_bytes=d["bytes"], algorithmic_flops=d["flops"],
+                            gbs=d["bytes"] / sec / 1e9, tflops=d["flops"] / sec / 1e12,
+                            roofline_us=1e6 * max(t_hbm, t_tc), frac=max(t_hbm, t_tc) / sec,
+                            bound="hbm" if t_hbm >= t_tc else "tensor")
+    top = max(detail, key=lambda n: detail[n]["ms"])
+    td = detail[top]
+    if td["bound"] == "hbm":
+        roof = dict(bound="hbm", achieved=td["gbs"], peak=peaks["hbm_gbs"], unit="GB/s", frac=td["gbs"] / peaks["hbm_gbs"])
+    else:
+        pk = peaks["bf16_tflops"] * (2.0 if top == "index" else 1.0)
+        roof = dict(bound="tensor", achieved=td["tflops"], peak=pk, unit="TFLOP/s", frac=td["tflops"] / pk)
+    roof["traffic"] = None
+    roof["kernel"] = top
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        cpu = dsa_cpu_baseline(inp, args.cpu_seconds)
+    sec = total_ms / 1e3
+    if rank == 0:
+        print(json.dumps(dict(
+            metric="sparse (DSA) decode steps/s: FP8 indexer + top-k + MLA decode over the selected tokens",
+            value=K / sec, unit="steps/s", n_gpus=1, steps=K, warmup=max(3, args.warmup), ms_per_step=total_ms / K,
+            higher_is_better=True, scaling="weak", vs_baseline=None, dtype="e4m3 indexer, bf16 decode",
+            data="synthetic",
+            config=dict(workload=dw.name, B=w.B, H=w.H, r=w.r, d_r=w.d_r, context=int(L), index_heads=dw.HI,
+                        index_dim=dw.dI, top_k=k, l2="inputs larger than L2: each step streams "
+                        f"{model['index']['bytes'] / 1e9:.2f} GB of indexer keys before the decode"),
+            tokens_per_s=K * w.B / sec, selected_tokens=model["selected"], context_tokens=model["tokens"],
+            roofline=roof, roofline_detail=dict(kernels=detail, peaks=peaks,
+                                                step_roofline_us=sum(d["roofline_us"] for d in detail.values())),
+            cpu_baseline=cpu, e2e=None, gpu_launches=4 * K, clocks=clocks)), flush=True)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -351,6 +497,9 @@ def main():
         return
     if args.op in ("absorb", "project"):
         head_gemm_arm(args, rank, local)
+        return
+    if args.op == "dsa":
+        dsa_arm(args, rank, local)
         return
 
     import torch

@@ -106,3 +106,57 @@ def head_gemm(x, w, y=None, stream=None):
     p = _b.HeadGemmParams(rows=rows, heads=H, k=k, n=n, reserved=0)
     _b.mla_head_gemm(p, x, w, y, stream=stream)
     return y
+
+
+def dsa_params_for(q_codes, k_codes, block_table, max_seq_len, top_k, causal=False) -> _b.DsaParams:
+    """mla_dsa_params_t from tensor shapes: q_codes [B, Sq, H^I, d^I], k_codes
+    [num_blocks, block_size, d^I], block_table [B, max_blocks]."""
+    B, Sq, HI, dI = q_codes.shape
+    nb, bs = k_codes.shape[0], k_codes.shape[1]
+    return _b.make_dsa_params(B, Sq, HI, dI, bs, nb, block_table.shape[1], max_seq_len, top_k, causal)
+
+
+def dsa_index(q_codes, q_scale, weights, k_codes, k_scale, block_table, seq_lens, max_seq_len, scores=None,
+              causal=False, stream=None):
+    """Lightning-indexer scores [B, Sq, max_seq_len] float32 (see mla_dsa_index). Code
+    tensors are uint8 (or float8_e4m3fn) e4m3 codes."""
+    import torch
+    p = dsa_params_for(q_codes, k_codes, block_table, max_seq_len, 1, causal)
+    if scores is None:
+        scores = torch.empty((q_codes.shape[0], q_codes.shape[1], max_seq_len), dtype=torch.float32,
+                             device=q_codes.device)
+    _b.mla_dsa_index(p, q_codes, q_scale, weights, k_codes, k_scale, block_table, seq_lens, scores, stream=stream)
+    return scores
+
+
+def dsa_topk(scores, seq_lens, top_k, causal=False, indices=None, counts=None, stream=None):
+    """Top-k positions per query row: (indices int32 [B, Sq, top_k] ascending, -1 padded;
+    counts int32 [B, Sq]) (see mla_dsa_topk)."""
+    import torch
+    B, Sq, max_seq_len = scores.shape
+    p = _b.make_dsa_params(B, Sq, 64, 128, 64, 1, max(1, (max_seq_len + 63) // 64), max_seq_len, top_k, causal)
+    if indices is None:
+        indices = torch.empty((B, Sq, top_k), dtype=torch.int32, device=scores.device)
+    if counts is None:
+        counts = torch.empty((B, Sq), dtype=torch.int32, device=scores.device)
+    _b.mla_dsa_topk(p, scores, seq_lens, indices, counts, stream=stream)
+    return indices, counts
+
+
+def sparse_decode(q_lat, q_rope, kv_cache, block_table, indices, counts, softmax_scale, out=None, lse=None,
+                  workspace=None, num_workers=0, stream=None):
+    """MLA decode over selected positions (q_len 1, bf16 cache): indices [B, top_k] (or
+    [B, 1, top_k]) int32, counts [B] (or [B, 1]) int32. Returns (out, lse)."""
+    import torch
+    p = params_for(q_lat, q_rope, kv_cache, block_table, softmax_scale, False, None, num_workers, "tcgen05")
+    top_k = indices.shape[-1]
+    dev = q_lat.device
+    if out is None:
+        out = torch.empty(q_lat.shape, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(q_lat.shape[:3], dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(_b.workspace_size(p), 1), dtype=torch.uint8, device=dev)
+    _b.mla_sparse_decode(p, top_k, q_lat, q_rope, kv_cache, block_table, indices, counts, out, lse, workspace,
+                         stream=stream)
+    return out, lse

@@ -26,7 +26,8 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "M
 EXPORTED = ("mla_decode_workspace_size", "mla_decode_resolve", "mla_decode", "mla_decode_timed",
             "mla_decode_host_io_workspace_size", "mla_decode_host_io", "mla_plan_host", "mla_plan_probe",
             "mla_get_device_status", "mla_status_string", "mla_abi_version", "mla_decode_noalloc",
-            "mla_decode_noalloc_max_workspace", "mla_cache_append", "mla_head_gemm")
+            "mla_decode_noalloc_max_workspace", "mla_cache_append", "mla_head_gemm", "mla_dsa_index",
+            "mla_dsa_topk", "mla_sparse_decode")
 
 
 class MlaError(RuntimeError):
@@ -59,6 +60,13 @@ class AppendParams(ctypes.Structure):
                 ("reserved", ctypes.c_int32)]
 
 
+class DsaParams(ctypes.Structure):
+    """mla_dsa_params_t."""
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "q_len", "index_heads", "index_dim", "block_size", "num_blocks", "max_blocks_per_seq",
+        "max_seq_len", "top_k", "causal", "reserved")]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is not built: run `python -m head_latent_attention_split_b200.build` "
@@ -83,6 +91,10 @@ def _load():
     L.mla_abi_version.argtypes = []
     L.mla_cache_append.argtypes = [ctypes.POINTER(AppendParams), vp, vp, vp, vp, vp, vp, vp, vp]
     L.mla_head_gemm.argtypes = [ctypes.POINTER(HeadGemmParams), vp, vp, vp, vp]
+    D = ctypes.POINTER(DsaParams)
+    L.mla_dsa_index.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.mla_dsa_topk.argtypes = [D, vp, vp, vp, vp, vp]
+    L.mla_sparse_decode.argtypes = [P, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     for name in EXPORTED:
         if not hasattr(L, name):
             raise ImportError(f"{LIB_PATH} lacks {name}: rebuild it")
@@ -275,4 +287,43 @@ def mla_head_gemm(p: HeadGemmParams, x, w, y, stream=None, check=True) -> int:
     st = lib.mla_head_gemm(ctypes.byref(p), _addr(x), _addr(w), _addr(y), _stream(stream))
     if check:
         _check(st, "mla_head_gemm")
+    return st
+
+
+def make_dsa_params(B, Sq, index_heads, index_dim, block_size, num_blocks, max_blocks_per_seq, max_seq_len, top_k,
+                    causal=False) -> DsaParams:
+    return DsaParams(batch=B, q_len=Sq, index_heads=index_heads, index_dim=index_dim, block_size=block_size,
+                     num_blocks=num_blocks, max_blocks_per_seq=max_blocks_per_seq, max_seq_len=max_seq_len,
+                     top_k=top_k, causal=int(bool(causal)), reserved=0)
+
+
+def mla_dsa_index(p: DsaParams, q_codes, q_scale, weights, k_codes, k_scale, block_table, seq_lens, scores,
+                  stream=None, check=True) -> int:
+    """Raw C-ABI call of the lightning indexer (device tensors or integer addresses)."""
+    st = lib.mla_dsa_index(ctypes.byref(p), _addr(q_codes), _addr(q_scale), _addr(weights), _addr(k_codes),
+                           _addr(k_scale), _addr(block_table), _addr(seq_lens), _addr(scores), _stream(stream))
+    if check:
+        _check(st, "mla_dsa_index")
+    return st
+
+
+def mla_dsa_topk(p: DsaParams, scores, seq_lens, indices, counts, stream=None, check=True) -> int:
+    """Raw C-ABI call of the top-k selection."""
+    st = lib.mla_dsa_topk(ctypes.byref(p), _addr(scores), _addr(seq_lens), _addr(indices), _addr(counts),
+                          _stream(stream))
+    if check:
+        _check(st, "mla_dsa_topk")
+    return st
+
+
+def mla_sparse_decode(p: Params, top_k: int, q_lat, q_rope, kv_cache, block_table, indices, counts, out, lse,
+                      workspace, workspace_bytes=None, stream=None, check=True) -> int:
+    """Raw C-ABI call of the decode over selected positions."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.mla_sparse_decode(ctypes.byref(p), int(top_k), _addr(q_lat), _addr(q_rope), _addr(kv_cache),
+                               _addr(block_table), _addr(indices), _addr(counts), _addr(out), _addr(lse),
+                               _addr(workspace), workspace_bytes, _stream(stream))
+    if check:
+        _check(st, "mla_sparse_decode")
     return st

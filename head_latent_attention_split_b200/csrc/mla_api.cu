@@ -431,6 +431,125 @@ mla_status_t mla_head_gemm(const mla_head_gemm_params_t* p, const void* x, const
   return mla::launch_head_gemm(a, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------- sparse attention
+namespace {
+mla_status_t check_dsa(const mla_dsa_params_t* p) {
+  if (!p) return MLA_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->q_len < 1 || p->index_heads < 1 || p->index_dim < 1 || p->block_size < 1 ||
+      p->num_blocks < 0 || p->max_blocks_per_seq < 1 || p->max_seq_len < 0 || p->top_k < 1 ||
+      (p->causal != 0 && p->causal != 1) || p->reserved != 0)
+    return MLA_ERR_INVALID_ARG;
+  if (p->batch > 0 && p->num_blocks < 1) return MLA_ERR_INVALID_ARG;
+  if (p->index_heads != mla::kDsaHeads || p->index_dim != mla::kDsaDim || p->block_size != 64)
+    return MLA_ERR_UNSUPPORTED;
+  if ((int64_t)p->batch * p->q_len > 65535) return MLA_ERR_UNSUPPORTED;   // one grid row per query row
+  if ((int64_t)p->max_blocks_per_seq * p->block_size > (1ll << 30)) return MLA_ERR_UNSUPPORTED;
+  if ((int64_t)p->num_blocks * p->block_size > (1ll << 31) - 1) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+mla::DsaArgs dsa_args(const mla_dsa_params_t* p, int* status) {
+  mla::DsaArgs a{};
+  a.B = p->batch;
+  a.Sq = p->q_len;
+  a.bs = p->block_size;
+  a.num_blocks = p->num_blocks;
+  a.max_blocks = p->max_blocks_per_seq;
+  a.max_seq_len = p->max_seq_len;
+  a.top_k = p->top_k;
+  a.causal = p->causal;
+  a.status = status;
+  return a;
+}
+}  // namespace
+
+mla_status_t mla_dsa_index(const mla_dsa_params_t* p, const void* q_codes, const float* q_scale,
+                           const float* weights, const void* k_codes, const float* k_scale,
+                           const int32_t* block_table, const int32_t* seq_lens, float* scores, void* stream) {
+  mla_status_t st = check_dsa(p);
+  if (st) return st;
+  if (p->batch == 0 || p->max_seq_len == 0) return MLA_OK;
+  if (!q_codes || !q_scale || !weights || !k_codes || !k_scale || !block_table || !seq_lens || !scores)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(q_codes, 16) || !aligned(k_codes, 16)) return MLA_ERR_ALIGNMENT;
+  const void* p4[] = {q_scale, weights, k_scale, block_table, seq_lens, scores};
+  for (const void* q : p4)
+    if (!aligned(q, 4)) return MLA_ERR_ALIGNMENT;
+  int* status = status_word(current_device());
+  if (!status) return MLA_ERR_CUDA;
+  mla::DsaArgs a = dsa_args(p, status);
+  a.q = (const uint8_t*)q_codes;
+  a.q_scale = q_scale;
+  a.w = weights;
+  a.k = (const uint8_t*)k_codes;
+  a.k_scale = k_scale;
+  a.block_table = block_table;
+  a.seq_lens = seq_lens;
+  a.scores = scores;
+  return mla::launch_dsa_index(a, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status_t mla_dsa_topk(const mla_dsa_params_t* p, const float* scores, const int32_t* seq_lens,
+                          int32_t* indices, int32_t* counts, void* stream) {
+  mla_status_t st = check_dsa(p);
+  if (st) return st;
+  if (p->batch == 0) return MLA_OK;
+  if (!scores || !seq_lens || !indices || !counts) return MLA_ERR_INVALID_ARG;
+  const void* p4[] = {scores, seq_lens, indices, counts};
+  for (const void* q : p4)
+    if (!aligned(q, 4)) return MLA_ERR_ALIGNMENT;
+  int* status = status_word(current_device());
+  if (!status) return MLA_ERR_CUDA;
+  mla::DsaArgs a = dsa_args(p, status);
+  a.scores = (float*)scores;
+  a.seq_lens = seq_lens;
+  a.indices = indices;
+  a.counts = counts;
+  return mla::launch_dsa_topk(a, (cudaStream_t)stream) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+mla_status_t mla_sparse_decode(const mla_decode_params_t* p, int32_t top_k, const void* q_lat,
+                               const void* q_rope, const void* kv_cache, const int32_t* block_table,
+                               const int32_t* indices, const int32_t* counts, void* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  int kernel = 0, W = 0;
+  mla_status_t st = resolve(p, &kernel, &W);
+  if (st) return st;
+  if (top_k < 1) return MLA_ERR_INVALID_ARG;
+  if (p->q_len != 1 || p->causal != 0 || p->cache_dtype != MLA_DTYPE_BF16 || kernel != MLA_KERNEL_TCGEN05)
+    return MLA_ERR_UNSUPPORTED;
+  if (p->batch == 0) return MLA_OK;
+  if (!q_lat || !q_rope || !kv_cache || !block_table || !indices || !counts || !out || !lse)
+    return MLA_ERR_INVALID_ARG;
+  const mla::WorkspaceLayout L = layout_for(p, W);
+  if (workspace_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (!workspace) return MLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q_lat, q_rope, kv_cache, block_table, out, lse};
+  for (const void* q : ptrs)
+    if (!aligned(q, 16)) return MLA_ERR_ALIGNMENT;
+  if (!aligned(indices, 4) || !aligned(counts, 4) || !aligned(workspace, 256)) return MLA_ERR_ALIGNMENT;
+  int* status = status_word(current_device());
+  if (!status) return MLA_ERR_CUDA;
+  mla::DecodeArgs a = make_args(p, W);
+  a.q_lat = q_lat;
+  a.q_rope = q_rope;
+  a.cache = kv_cache;
+  a.block_table = block_table;
+  a.seq_lens = counts;   // each sequence's length is its list's count
+  a.sel_idx = indices;
+  a.top_k = top_k;
+  a.out = out;
+  a.lse = lse;
+  char* ws = (char*)workspace;
+  a.meta = (int32_t*)(ws + L.meta_off);
+  a.lse_part = (float*)(ws + L.lse_off);
+  a.o_part = (float*)(ws + L.o_off);
+  a.status = status;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (mla::launch_tc_decode(a, s) != cudaSuccess) return MLA_ERR_CUDA;
+  return mla::launch_combine(a, s) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 mla_status_t mla_get_device_status(void* stream, int32_t* device_status) {
   if (!device_status) return MLA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MLA_ERR_CUDA;

@@ -29,7 +29,9 @@ struct DecodeArgs {
   const uint16_t* k_rope;      // E4M3 only: bf16 [nb, bs, d_r]
   const float* kv_scale;       // E4M3 only: [nb, bs]
   const int32_t* block_table;  // [B, max_blocks]
-  const int32_t* seq_lens;     // [B]
+  const int32_t* seq_lens;     // [B]; sparse decode: the selected token counts
+  const int32_t* sel_idx;      // sparse decode only: [B, top_k] selected positions, else null
+  int top_k;                   // sparse decode only: row stride of sel_idx
   void* out;                   // [B, Sq, H, r] out_dtype
   float* lse;                  // [B, Sq, H]
   // workspace
@@ -96,5 +98,25 @@ struct GemmArgs {
   int* status;
 };
 cudaError_t launch_head_gemm(const GemmArgs& a, cudaStream_t s);
+
+// Sparse attention side kernels (mla_dsa.cu): the FP8 lightning indexer and top-k.
+constexpr int kDsaHeads = 64;    // indexer heads H^I of the tensor path
+constexpr int kDsaDim = 128;     // indexer width d^I of the tensor path
+struct DsaArgs {
+  int B, Sq, bs, num_blocks, max_blocks, max_seq_len, top_k, causal;
+  const uint8_t* q;            // [B, Sq, 64, 128] e4m3
+  const float* q_scale;        // [B, Sq, 64]
+  const float* w;              // [B, Sq, 64]
+  const uint8_t* k;            // [num_blocks, bs, 128] e4m3
+  const float* k_scale;        // [num_blocks, bs]
+  const int32_t* block_table;  // [B, max_blocks]
+  const int32_t* seq_lens;     // [B]
+  float* scores;               // [B, Sq, max_seq_len]
+  int32_t* indices;            // [B, Sq, top_k]
+  int32_t* counts;             // [B, Sq]
+  int* status;
+};
+cudaError_t launch_dsa_index(const DsaArgs& a, cudaStream_t s);
+cudaError_t launch_dsa_topk(const DsaArgs& a, cudaStream_t s);
 
 }  // namespace mla

@@ -47,6 +47,13 @@
 //    and epilogue, warp 8 TMA producer, warp 9 TMEM allocator and single-thread MMA
 //    issuer, warps 10-11 FP8 converters; mbarrier pipelines between them. Every wait is
 //    bounded (timeout -> MLA_ERR_TIMEOUT, clean exit).
+//  * Sparse decode (DeepSeek Sparse Attention: "TransMLA & Sparse Latent Attention"
+//    lesson, Chapter 7 "DSA runs in MLA's MQA mode"): the same kernel over each
+//    sequence's list of selected positions instead of its whole length. The per-sequence
+//    length is the list's count, and tile t holds list entries [64 t, 64 t + 64); the
+//    producer warp maps them through the block table and fetches the 64 token rows of
+//    the CTA's channel slice with TMA row gathers (four rows per load), into the same
+//    swizzled stage layout. Entries past the count read as zeros.
 // The work split over workers (CTA pairs) is the flat block list plan of mla_device.cuh.
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -158,7 +165,7 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two_codes) {
   return __half22float2(*reinterpret_cast<const __half2*>(&h2));
 }
 
-template <bool kFp8>
+template <bool kFp8, bool kSparse>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(), 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_sc,
@@ -228,7 +235,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
   const uint32_t tmem = ctl.tmem_base;
   const WorkerPlan plan = ctl.plan;
 
-  if (warp == kProducerWarp) {
+  if (kSparse && warp == kProducerWarp) {
+    // ------------------------------------------------------------------ gather producer (sparse)
+    // Lanes map the 64 listed positions of a tile to cache rows (two each); lane l < 16
+    // then loads rows 4 l .. 4 l + 3 of every channel chunk with one row gather each.
+    SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
+    Segment sg;
+    uint32_t g = 0, seg = 0;
+    bool ok = true;
+    const int oob_row = a.num_blocks * kBS;   // past the last row: the load fills zeros
+    while (ok && it.next(sg)) {
+      if (lane == 0) {
+        ok = mbar_wait<false>(smem_u32(&ctl.q_empty), (seg & 1) ^ 1, abort, timeout_ns);
+        if (ok) {
+          const uint32_t qbar = smem_u32(&ctl.q_full);
+          mbar_arrive_expect_tx(qbar, kQRope);
+          tma_load_3d(sQr, &tm_qr, qbar, 32 * rank, rg * kRows, sg.b);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      for (int tile = sg.tile_begin; tile < sg.tile_end; ++tile, ++g) {
+        int rw[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int j = tile * kBS + 32 * hh + lane;   // list entry
+          int row = oob_row;
+          if (j < sg.Lc) {
+            const int t = __ldg(a.sel_idx + (size_t)sg.b * a.top_k + j);
+            const int blk = (t >= 0 && t < cap) ? __ldg(a.block_table + (size_t)sg.b * a.max_blocks + t / kBS) : -1;
+            if (blk >= 0 && blk < a.num_blocks)
+              row = blk * kBS + t % kBS;
+            else
+              set_status(a.status, MLA_ERR_BAD_BLOCK_ID);
+          }
+          rw[hh] = row;
+        }
+        int r4[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int i = 4 * lane + m;   // token row of the tile (meaningful for lanes < 16)
+          const int v0 = __shfl_sync(0xffffffffu, rw[0], i & 31);
+          const int v1 = __shfl_sync(0xffffffffu, rw[1], i & 31);
+          r4[m] = i < 32 ? v0 : v1;
+        }
+        const uint32_t st = g % kStages, ph = (g / kStages) & 1;
+        if (lane == 0) ok = mbar_wait<false>(smem_u32(&ctl.kv_empty[st]), ph ^ 1, abort, timeout_ns);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        const uint32_t bar = smem_u32(&ctl.kv_full[st]);
+        const uint32_t base = sKv + st * kStageBytes;
+        if (lane == 0) mbar_arrive_expect_tx(bar, kStageBytes);
+        __syncwarp();
+        if (lane < 16) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tma_gather4(base + c * kKvLatChunk + lane * 512, &tm_kv, bar, 256 * rank + 64 * c, r4);
+          tma_gather4(base + 4 * kKvLatChunk + lane * 256, &tm_kr, bar, kR + 32 * rank, r4);
+        }
+      }
+      ++seg;
+    }
+    if (lane == 0) {
+      int dummy = 0;
+      for (uint32_t i = 0; i < kStages && i < g; ++i) {
+        const uint32_t gl = g - 1 - i;
+        mbar_wait<false>(smem_u32(&ctl.kv_full[gl % kStages]), (gl / kStages) & 1, &dummy, timeout_ns);
+      }
+      if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
+    }
+  } else if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
@@ -870,6 +945,20 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D tensor map with a one-row box, for row gathers: dims (inner, rows), row stride s1.
+bool make_map_2d_rows(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t s1, uint32_t b0,
+                      CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {s1};
+  const cuuint32_t box[2] = {b0, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int row_groups(int rows) { return (rows + kRows - 1) / kRows; }
 
 }  // namespace
@@ -892,8 +981,15 @@ cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
   CUtensorMap tqr, tkv, tkr, tsc;
   const uint64_t rows = (uint64_t)a.rows;
   const bool fp8 = a.cache_dtype == kE4M3;
+  const bool sparse = a.sel_idx != nullptr;
+  if (sparse && (fp8 || a.Sq != 1 || a.causal)) return cudaErrorInvalidValue;
   bool ok = make_map_3d(&tqr, a.q_rope, kDR, rows, a.B, kDR * 2, rows * kDR * 2, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B);
-  if (fp8) {
+  if (sparse) {
+    // the cache as rows [num_blocks * 64][576] bf16: 64-channel latent boxes, 32-channel RoPE boxes
+    const uint64_t nrows = (uint64_t)a.num_blocks * kBS;
+    ok = ok && make_map_2d_rows(&tkv, a.cache, kR + kDR, nrows, (kR + kDR) * 2, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map_2d_rows(&tkr, a.cache, kR + kDR, nrows, (kR + kDR) * 2, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  } else if (fp8) {
     // codes [num_blocks][64][512] e4m3 (256-byte boxes, no swizzle), RoPE keys [num_blocks][64][64] bf16
     ok = ok &&
          make_map_3d(&tkv, a.cache, kR, kBS, a.num_blocks, kR, (uint64_t)kBS * kR, 256, kBS, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -910,26 +1006,32 @@ cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
                      kBS, CU_TENSOR_MAP_SWIZZLE_64B);
   }
   if (!ok) return cudaErrorInvalidValue;
-  if (!fp8) tsc = tkr;   // unused by the bf16 kernel
-  static std::once_flag attr_once[2][64];
+  if (!fp8) tsc = tkr;   // unused by the bf16 kernels
+  static std::once_flag attr_once[3][64];
   int dev = 0;
   cudaGetDevice(&dev);
+  const int variant = sparse ? 2 : fp8 ? 1 : 0;
   cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once[fp8 ? 1 : 0][dev & 63], [&] {
-    attr_err = fp8 ? cudaFuncSetAttribute(tc_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          Geo<true>::kSmemBytes)
-                   : cudaFuncSetAttribute(tc_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          Geo<false>::kSmemBytes);
+  std::call_once(attr_once[variant][dev & 63], [&] {
+    attr_err = variant == 1 ? cudaFuncSetAttribute(tc_decode_kernel<true, false>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, Geo<true>::kSmemBytes)
+               : variant == 2 ? cudaFuncSetAttribute(tc_decode_kernel<false, true>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, Geo<false>::kSmemBytes)
+                              : cudaFuncSetAttribute(tc_decode_kernel<false, false>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, Geo<false>::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
   const uint64_t timeout_ns = 2000000000ull;
   const dim3 grid(2 * a.W * n_rg);
-  if (fp8)
-    tc_decode_kernel<true><<<grid, threads_for<true>(), Geo<true>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a, n_rg,
-                                                                                    timeout_ns);
+  if (variant == 1)
+    tc_decode_kernel<true, false><<<grid, threads_for<true>(), Geo<true>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a, n_rg,
+                                                                                           timeout_ns);
+  else if (variant == 2)
+    tc_decode_kernel<false, true><<<grid, threads_for<false>(), Geo<false>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a,
+                                                                                             n_rg, timeout_ns);
   else
-    tc_decode_kernel<false><<<grid, threads_for<false>(), Geo<false>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a, n_rg,
-                                                                                       timeout_ns);
+    tc_decode_kernel<false, false><<<grid, threads_for<false>(), Geo<false>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a,
+                                                                                              n_rg, timeout_ns);
   return cudaGetLastError();
 }
 

@@ -276,6 +276,65 @@ typedef struct {
 mla_status_t mla_head_gemm(const mla_head_gemm_params_t* params, const void* x, const void* w, void* y,
                            void* stream);
 
+/* ------------------------------------------------------------------ sparse attention (DSA)
+ *
+ * DeepSeek Sparse Attention on the same paged cache ("TransMLA & Sparse Latent Attention"
+ * lesson, Chapter 6 "The lightning indexer" and "Fine-grained token selection"; Chapter 7
+ * "The indexer keeps its own small cache" and "DSA runs in MLA's MQA mode"). One sparse
+ * decode step is three calls on one stream:
+ *
+ *   mla_dsa_index   scores[b,s,t] = sum_j w[b,s,j] * ReLU( q_j . k_t ) for every token t
+ *                   query row (b, s) sees (the decode's causal rule), j < index_heads;
+ *                   q_j = e4m3(q_codes[b,s,j,:]) * q_scale[b,s,j],
+ *                   k_t = e4m3(k_codes[slot(t),:]) * k_scale[slot(t)], slot(t) through the
+ *                   block table. Entries t >= that count are not written.
+ *   mla_dsa_topk    for each row, the positions of its top_k highest scores (all of them
+ *                   when it sees top_k or fewer tokens), ascending, -1 past the count;
+ *                   equal scores at the cut go to the lower positions (-0 equals +0).
+ *                   counts[b,s] = min(seen, top_k).
+ *   mla_sparse_decode  the decode above over each sequence's selected positions only
+ *                   (q_len 1, bf16 cache, tensor-core kernel): row (b, 0, h) attends
+ *                   exactly tokens indices[b, 0 .. counts[b]).
+ *
+ * Tensors (device, contiguous): q_codes uint8 [B, Sq, index_heads, index_dim] and
+ * k_codes uint8 [num_blocks, block_size, index_dim] (the indexer's key side-cache, paged
+ * like the latent cache), both 16-byte aligned; q_scale, weights f32 [B, Sq, index_heads];
+ * k_scale f32 [num_blocks, block_size] (scales >= 0); scores f32 [B, Sq, max_seq_len];
+ * indices int32 [B, Sq, top_k]; counts int32 [B, Sq]. The tensor path has index_heads 64,
+ * index_dim 128, block_size 64 (MLA_ERR_UNSUPPORTED otherwise). A seq_len above
+ * max_seq_len or the block table's capacity sets MLA_ERR_BAD_SEQ_LEN on the device (that
+ * row is skipped); a block id out of range sets MLA_ERR_BAD_BLOCK_ID (its tokens score
+ * NaN; in the sparse decode they read as zeros). Positions handed to the sparse decode
+ * must be below their sequence's length. Asynchronous, allocates nothing. */
+typedef struct {
+  int32_t batch;               /* B */
+  int32_t q_len;               /* Sq */
+  int32_t index_heads;         /* H^I (64) */
+  int32_t index_dim;           /* d^I (128) */
+  int32_t block_size;          /* 64 */
+  int32_t num_blocks;
+  int32_t max_blocks_per_seq;  /* row stride of block_table */
+  int32_t max_seq_len;         /* row stride of scores; >= every seq_len */
+  int32_t top_k;               /* k (2048 in DeepSeek-V3.2) */
+  int32_t causal;              /* 0 or 1, as in the decode */
+  int32_t reserved;            /* must be 0 */
+} mla_dsa_params_t;
+
+mla_status_t mla_dsa_index(const mla_dsa_params_t* params, const void* q_codes, const float* q_scale,
+                           const float* weights, const void* k_codes, const float* k_scale,
+                           const int32_t* block_table, const int32_t* seq_lens, float* scores, void* stream);
+
+mla_status_t mla_dsa_topk(const mla_dsa_params_t* params, const float* scores, const int32_t* seq_lens,
+                          int32_t* indices, int32_t* counts, void* stream);
+
+/* The decode's params (q_len 1, causal 0, BF16 cache, kernel AUTO or TCGEN05) and
+ * workspace (mla_decode_workspace_size of the same params). indices [B, top_k] int32,
+ * counts [B] int32, device. */
+mla_status_t mla_sparse_decode(const mla_decode_params_t* params, int32_t top_k, const void* q_lat,
+                               const void* q_rope, const void* kv_cache, const int32_t* block_table,
+                               const int32_t* indices, const int32_t* counts, void* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
 /* MLA_DECODE_ABI_VERSION of the loaded library. */
 int32_t mla_abi_version(void);
 

@@ -201,3 +201,67 @@ def test_append_rejects_bad_arguments_on_host(m, bad):
 
 def test_append_batch_zero_is_a_noop(m):
     assert _append(m, B=0, c_new=None, kv_cache=None, block_table=None, seq_lens=None) == 0
+
+
+# ----------------------------------------------------------------------------- sparse attention
+def _dsa(m, fn="index", **kw):
+    from head_latent_attention_split_b200 import binding
+    args = dict(B=2, Sq=1, index_heads=64, index_dim=128, block_size=64, num_blocks=8, max_blocks_per_seq=4,
+                max_seq_len=256, top_k=64, causal=False)
+    reserved = kw.pop("reserved", 0)
+    causal_raw = kw.pop("causal_raw", None)
+    ptr_names = ("q_codes", "q_scale", "weights", "k_codes", "k_scale", "block_table", "seq_lens", "scores",
+                 "indices", "counts")
+    ptrs = {k: kw.pop(k, FAKE) for k in ptr_names}
+    args.update(kw)
+    p = binding.make_dsa_params(**args)
+    p.reserved = reserved
+    if causal_raw is not None:
+        p.causal = causal_raw
+    if fn == "index":
+        return binding.mla_dsa_index(p, ptrs["q_codes"], ptrs["q_scale"], ptrs["weights"], ptrs["k_codes"],
+                                     ptrs["k_scale"], ptrs["block_table"], ptrs["seq_lens"], ptrs["scores"],
+                                     stream=0, check=False)
+    return binding.mla_dsa_topk(p, ptrs["scores"], ptrs["seq_lens"], ptrs["indices"], ptrs["counts"], stream=0,
+                                check=False)
+
+
+@pytest.mark.parametrize("fn", ["index", "topk"])
+@pytest.mark.parametrize("bad,code", [(dict(Sq=0), 1), (dict(top_k=0), 1), (dict(causal_raw=2), 1), (dict(reserved=1), 1),
+                                      (dict(max_seq_len=-1), 1), (dict(num_blocks=0), 1), (dict(index_heads=32), 2),
+                                      (dict(index_dim=64), 2), (dict(block_size=32), 2), (dict(B=70000), 2),
+                                      (dict(scores=None), 1)])
+def test_dsa_rejects_bad_arguments_on_host(m, fn, bad, code):
+    assert _dsa(m, fn, **bad) == code
+
+
+def test_dsa_null_and_alignment_checks(m):
+    assert _dsa(m, "index", q_codes=None) == 1
+    assert _dsa(m, "index", k_codes=FAKE + 8) == 3           # TMA source: 16-byte aligned
+    assert _dsa(m, "topk", indices=None) == 1
+    assert _dsa(m, "topk", counts=FAKE + 2) == 3
+    assert _dsa(m, "index", B=0, q_codes=None) == 0           # nothing to do
+    assert _dsa(m, "topk", B=0, scores=None) == 0
+
+
+def _sparse(m, **kw):
+    from head_latent_attention_split_b200 import binding
+    base = dict(B=2, Sq=1, H=128, r=512, d_r=64, block_size=64, num_blocks=8, max_blocks_per_seq=4, q_dtype=1,
+                cache_dtype=1, out_dtype=1, causal=False, softmax_scale=0.07, num_workers=4, kernel="tcgen05")
+    top_k = kw.pop("top_k", 64)
+    ptr_names = ("q_lat", "q_rope", "kv_cache", "block_table", "indices", "counts", "out", "lse", "workspace")
+    ptrs = {k: kw.pop(k, FAKE) for k in ptr_names}
+    ws_bytes = kw.pop("workspace_bytes", 1 << 30)
+    base.update(kw)
+    p = m.make_params(**base)
+    return binding.mla_sparse_decode(p, top_k, ptrs["q_lat"], ptrs["q_rope"], ptrs["kv_cache"], ptrs["block_table"],
+                                     ptrs["indices"], ptrs["counts"], ptrs["out"], ptrs["lse"], ptrs["workspace"],
+                                     workspace_bytes=ws_bytes, stream=0, check=False)
+
+
+@pytest.mark.parametrize("bad,code", [(dict(Sq=2), 2), (dict(causal=True), 2), (dict(cache_dtype=2), 2),
+                                      (dict(kernel="simt"), 2), (dict(top_k=0), 1), (dict(indices=None), 1),
+                                      (dict(counts=None), 1), (dict(q_rope=None), 1), (dict(workspace_bytes=16), 4),
+                                      (dict(q_lat=FAKE + 8), 3), (dict(indices=FAKE + 2), 3)])
+def test_sparse_decode_rejects_bad_arguments_on_host(m, bad, code):
+    assert _sparse(m, **bad) == code
