@@ -471,8 +471,8 @@ mla_status_t mla_dsa_index(const mla_dsa_params_t* p, const void* q_codes, const
   if (p->batch == 0 || p->max_seq_len == 0) return MLA_OK;
   if (!q_codes || !q_scale || !weights || !k_codes || !k_scale || !block_table || !seq_lens || !scores)
     return MLA_ERR_INVALID_ARG;
-  if (!aligned(q_codes, 16) || !aligned(k_codes, 16)) return MLA_ERR_ALIGNMENT;
-  const void* p4[] = {q_scale, weights, k_scale, block_table, seq_lens, scores};
+  if (!aligned(q_codes, 16) || !aligned(k_codes, 16) || !aligned(k_scale, 16)) return MLA_ERR_ALIGNMENT;
+  const void* p4[] = {q_scale, weights, block_table, seq_lens, scores};
   for (const void* q : p4)
     if (!aligned(q, 4)) return MLA_ERR_ALIGNMENT;
   int* status = status_word(current_device());

@@ -299,7 +299,8 @@ mla_status_t mla_head_gemm(const mla_head_gemm_params_t* params, const void* x, 
  * Tensors (device, contiguous): q_codes uint8 [B, Sq, index_heads, index_dim] and
  * k_codes uint8 [num_blocks, block_size, index_dim] (the indexer's key side-cache, paged
  * like the latent cache), both 16-byte aligned; q_scale, weights f32 [B, Sq, index_heads];
- * k_scale f32 [num_blocks, block_size] (scales >= 0); scores f32 [B, Sq, max_seq_len];
+ * k_scale f32 [num_blocks, block_size], 16-byte aligned (scales >= 0: the kernel folds them
+ * out of the ReLU); scores f32 [B, Sq, max_seq_len];
  * indices int32 [B, Sq, top_k]; counts int32 [B, Sq]. The tensor path has index_heads 64,
  * index_dim 128, block_size 64 (MLA_ERR_UNSUPPORTED otherwise). A seq_len above
  * max_seq_len or the block table's capacity sets MLA_ERR_BAD_SEQ_LEN on the device (that

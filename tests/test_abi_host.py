@@ -237,7 +237,8 @@ def test_dsa_rejects_bad_arguments_on_host(m, fn, bad, code):
 
 def test_dsa_null_and_alignment_checks(m):
     assert _dsa(m, "index", q_codes=None) == 1
-    assert _dsa(m, "index", k_codes=FAKE + 8) == 3           # TMA source: 16-byte aligned
+    assert _dsa(m, "index", k_codes=FAKE + 8) == 3           # TMA sources: 16-byte aligned
+    assert _dsa(m, "index", k_scale=FAKE + 4) == 3
     assert _dsa(m, "topk", indices=None) == 1
     assert _dsa(m, "topk", counts=FAKE + 2) == 3
     assert _dsa(m, "index", B=0, q_codes=None) == 0           # nothing to do

@@ -174,7 +174,8 @@ def topk_case(seed, rows, L, tie_levels=None):
 
 
 @pytest.mark.parametrize("L,top_k,ties", [(70000, 2048, None), (70000, 2048, 50), (5000, 1, None), (5000, 4999, 7),
-                                          (9000, 4096, 3), (300, 512, None)])
+                                          (9000, 4096, 3), (300, 512, None),
+                                          (140000, 2048, 9)])   # slices beyond the register-resident size
 def test_topk_bit_exact(L, top_k, ties):
     mla = _mla()
     s = topk_case(L + top_k, 4, L, ties)
