@@ -75,15 +75,21 @@ def load_peaks():
 # only holds for the kernel sources it was taken on, keyed here by their SHA-256 prefix; for
 # any other source the bench reports traffic as null.
 MEASURED_TRAFFIC = {
-    "423e4906d137dc85": {"deepseek_v3": (304.118272e6 + 5.891840e6) / 262144,
-                 "fp8_cache": (169.787904e6 + 5.152768e6) / 262144},
+    "524335d759a92050": {"deepseek_v3": (304.125184e6 + 4.850944e6) / 262144,
+                         "fp8_cache": (169.770496e6 + 5.082368e6) / 262144},
 }
 KERNEL_SOURCES = ("mla_tc.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.h", "mla_tc.h")
+# The same for the sparse step's indexer (dram bytes per context token, batch 8 of the
+# 128K workload), keyed by the sources of mla_dsa.cu and its headers.
+DSA_TRAFFIC = {
+    "4062b4c681eeff4c": {"dsa_v32": (138.621440e6 + 5.537536e6) / (8 * 131072)},
+}
+DSA_SOURCES = ("mla_dsa.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.h")
 
 
-def kernel_source_hash():
+def kernel_source_hash(files=KERNEL_SOURCES):
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in files:
         with open(os.path.join(ROOT, "head_latent_attention_split_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -463,7 +469,8 @@ def dsa_arm(args, rank, local):
     else:
         pk = peaks["bf16_tflops"] * (2.0 if top == "index" else 1.0)
         roof = dict(bound="tensor", achieved=td["tflops"], peak=pk, unit="TFLOP/s", frac=td["tflops"] / pk)
-    roof["traffic"] = None
+    per_tok = DSA_TRAFFIC.get(kernel_source_hash(DSA_SOURCES), {}).get(W.DSA_BY_NAME[args.dsa_workload].name)
+    roof["traffic"] = per_tok * model["tokens"] if (per_tok is not None and top == "index") else None
     roof["kernel"] = top
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
