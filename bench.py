@@ -82,7 +82,7 @@ KERNEL_SOURCES = ("mla_tc.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.
 # The same for the sparse step's indexer (dram bytes per context token, batch 8 of the
 # 128K workload), keyed by the sources of mla_dsa.cu and its headers.
 DSA_TRAFFIC = {
-    "4062b4c681eeff4c": {"dsa_v32": (138.621440e6 + 5.537536e6) / (8 * 131072)},
+    "af77376c40dcd323": {"dsa_v32": (138.621952e6 + 4.314624e6) / (8 * 131072)},
 }
 DSA_SOURCES = ("mla_dsa.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.h")
 

@@ -4,9 +4,9 @@
 //
 // Indexer: I_t = sum_j w_j * ReLU(q_j . k_t) for every token t a query row may see, with
 // H^I = 64 heads of width d^I = 128 stored as e4m3 codes with one fp32 scale per vector
-// (q per head, k per cached token). A persistent CTA per SM walks a contiguous range of
+// (q per head, k per cached token). Persistent CTAs (two per SM) walk contiguous ranges of
 // (query row, 128-token tile) items. TMA brings each tile's key codes (two cache blocks,
-// 128-byte swizzled) through an 8-stage ring and the row's 64 x 128 query codes; one
+// 128-byte swizzled) and key scales through a stage ring and the row's 64 x 128 query codes; one
 // thread issues tcgen05 MMAs of kind::f8f6f4 with the tokens as M = 128 and the heads as
 // N = 64 (K = 4 x 32 codes) into a ring of TMEM accumulators, so every TMEM lane holds one
 // token's 64 head dots and the thread reading it finishes that token alone: scale, ReLU,
@@ -34,17 +34,19 @@ namespace {
 using namespace ptx;
 
 // ------------------------------------------------------------------------------ indexer
-// Persistent: one CTA per SM walks a contiguous range of (query row, 128-token tile) items.
-// Warp 4 produces (TMA: the tile's two cache blocks and their key scales into a 10-stage
+// Persistent: two CTAs per SM, each walking a contiguous range of (query row, 128-token tile)
+// items. Warp 4 produces (TMA: the tile's two cache blocks and their key scales into a 5-stage
 // ring, the row's query into one of two slots when the row changes), warp 5 allocates TMEM
-// and issues the MMAs into a ring of four 64-column accumulators, and two groups of four
-// warps finish the tokens (thread = token), warps 0-3 the even items and warps 6-9 the odd
-// ones, so that one item's TMEM read and sum overlap the other's.
+// and issues the MMAs into a ring of four 64-column accumulators, and warps 0-3 finish the
+// tokens (thread = token). The per-tile handoff is latency-bound, so two independent CTAs per
+// SM keep twice the tiles in flight (a second epilogue group in one CTA, kIGroups = 2, does not).
 constexpr int kITok = 128;                        // tokens per tile = MMA M
 constexpr int kIBlk = 64;                         // tokens per cache block
-constexpr int kIStages = 10;
+constexpr int kIStages = 5;                // TMA ring depth
+constexpr int kIGroups = 1;                // epilogue warp groups (items alternate between them when 2)
+constexpr int kICtasPerSm = 2;             // two independent pipelines per SM (TMEM: 2 x 256 columns)
 constexpr int kIAcc = 4;
-constexpr int kIThreads = 320;
+constexpr int kIThreads = 192 + 128 * (kIGroups - 1);
 constexpr int kIProducer = 4, kIMma = 5;   // epilogue groups: warps 0-3 (even items), 6-9 (odd items)
 constexpr uint32_t kIKTile = kITok * kDsaDim;     // 16 KB of key codes
 constexpr uint32_t kIQ = kDsaHeads * kDsaDim;     // 8 KB of query codes
@@ -61,12 +63,13 @@ struct IdxCtl {
   uint32_t valid[kIStages];             // per stage: bit h set = block h of the tile was loaded
   float wq[2][kDsaHeads];               // per query slot: weight x query scale of each head
 };
-constexpr uint32_t kIOffS = kIStages * kIKTile;                 // key scales ring
-constexpr uint32_t kIOffQ = kIOffS + kIStages * kIScales;      // two query slots
-constexpr uint32_t kIOffCtl = kIOffQ + 2 * kIQ;
+constexpr uint32_t kIOffQ = kIStages * kIKTile;                 // two query slots
+constexpr uint32_t kIOffS = kIOffQ + 2 * kIQ;                    // key scales ring
+constexpr uint32_t kIOffCtl = kIOffS + kIStages * kIScales;
 static_assert(kIOffQ % 1024 == 0, "query slots need 1024-byte alignment");
 constexpr uint32_t kISmem = kIOffCtl + 2048 + 1024;   // + control + alignment
-static_assert(sizeof(IdxCtl) <= 2048 && kISmem <= 232448, "indexer shared memory");
+static_assert(sizeof(IdxCtl) <= 2048 && kICtasPerSm * (kISmem + 1024) <= 232448, "indexer shared memory");
+static_assert(kICtasPerSm * kIAcc * kDsaHeads <= 512, "TMEM columns per SM");
 
 // tokens query row r sees; a bad seq_len flags the status and counts as 0
 __device__ __forceinline__ int row_tokens(const DsaArgs& a, int r, bool report) {
@@ -100,7 +103,7 @@ struct ItemWalk {
   }
 };
 
-__global__ void __launch_bounds__(kIThreads, 1)
+__global__ void __launch_bounds__(kIThreads, kICtasPerSm)
     dsa_index_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_s, const DsaArgs a, const uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
@@ -148,7 +151,7 @@ __global__ void __launch_bounds__(kIThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&ctl.q_full[i]), 1);
-      mbar_init(smem_u32(&ctl.q_empty[i]), 1 + 8);   // the MMAs of the row and each epilogue warp
+      mbar_init(smem_u32(&ctl.q_empty[i]), 1 + 4 * kIGroups);   // the MMAs of the row and each epilogue warp
     }
     ctl.abort = 0;
     fence_mbarrier_init_cluster();
@@ -298,7 +301,7 @@ __global__ void __launch_bounds__(kIThreads, 1)
                                                       timeout_ns) && !*abort);
         if (!ok) break;
       }
-      if ((i & 1) != grp) continue;   // the other group's item
+      if (kIGroups == 2 && (i & 1) != grp) continue;   // the other group's item
       const float* wq = ctl.wq[rs & 1];
       const int t = it.j * kITok + tr;
       const uint32_t st = i % kIStages, ac = i % kIAcc;
@@ -622,9 +625,9 @@ cudaError_t launch_dsa_index(const DsaArgs& a, cudaStream_t s) {
     if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms[dev & 63], cudaDevAttrMultiProcessorCount, dev);
   });
   if (err != cudaSuccess) return err;
-  // one CTA per SM, fewer when there are fewer tiles than SMs
+  // kICtasPerSm CTAs per SM, fewer when there are fewer tiles
   const long long tiles_max = (long long)R * ((a.max_seq_len + kITok - 1) / kITok);
-  const int grid = (int)std::min<long long>(std::max(sms[dev & 63], 1), std::max(tiles_max, 1ll));
+  const int grid = (int)std::min<long long>((long long)kICtasPerSm * std::max(sms[dev & 63], 1), std::max(tiles_max, 1ll));
   dsa_index_kernel<<<grid, kIThreads, kISmem, s>>>(tq, tk, ts, a, 2000000000ull);
   return cudaGetLastError();
 }

@@ -333,3 +333,63 @@ def test_full_size_sampled_rows(full):
                                       inp["block_table"][b:b + 1], inp["seq_lens"][b:b + 1], w.scale,
                                       lst[b:b + 1].reshape(1, 1, k), cnts[b:b + 1].reshape(1, 1))
         compare(out[b:b + 1], lse[b:b + 1], ro, rl, TOL[W.BF16], f"full-size sparse decode b={b}")
+
+
+# ----------------------------------------------------------------------------- error paths
+def test_index_bad_block_id_and_seq_len_set_status(small):
+    """A block id outside [0, num_blocks) marks its tokens NaN and sets MLA_ERR_BAD_BLOCK_ID; a
+    seq_len above max_seq_len skips the row and sets MLA_ERR_BAD_SEQ_LEN. Neither loads past the
+    cache (the bad block is not fetched)."""
+    torch = _torch()
+    mla = _mla()
+    inp = dict(small)
+    bt = inp["block_table"].copy()
+    bt[1, 3] = inp["num_blocks"] + 7               # tokens [192, 256) of sequence 1
+    inp["block_table"] = bt
+    w = inp["workload"]
+    L = inp["max_seq_len"]
+    scores = torch.full((w.B, 1, L), -12345.0, dtype=torch.float32, device="cuda")
+    mla.dsa_index(_dev(inp["iq_codes"]), _dev(inp["iq_scale"]), _dev(inp["iw"]), _dev(inp["ik_codes"]),
+                  _dev(inp["ik_scale"]), _dev(bt), _dev(inp["seq_lens"]), L, scores=scores)
+    torch.cuda.synchronize()
+    assert mla.device_status() == 6                 # MLA_ERR_BAD_BLOCK_ID (read and cleared)
+    assert mla.device_status() == 0
+    g = scores.cpu().numpy()
+    assert np.isnan(g[1, 0, 192:256]).all() and np.isfinite(g[1, 0, :192]).all()
+    assert np.isfinite(g[1, 0, 256:4100]).all() and np.isfinite(g[0, 0, :300]).all()
+    sl = inp["seq_lens"].copy()
+    sl[2] = L + 1                                   # longer than the score rows
+    scores.fill_(-12345.0)
+    mla.dsa_index(_dev(inp["iq_codes"]), _dev(inp["iq_scale"]), _dev(inp["iw"]), _dev(inp["ik_codes"]),
+                  _dev(inp["ik_scale"]), _dev(small["block_table"]), _dev(sl), L, scores=scores)
+    idx, cnt = mla.dsa_topk(scores, _dev(sl), 64)
+    torch.cuda.synchronize()
+    assert mla.device_status() == 7                 # MLA_ERR_BAD_SEQ_LEN
+    g = scores.cpu().numpy()
+    assert (g[2] == -12345.0).all() and np.isfinite(g[0, 0, :300]).all()
+    assert cnt.cpu().numpy()[2, 0] == 0 and (idx.cpu().numpy()[2] == -1).all()
+
+
+def test_sparse_decode_bad_position_sets_status(small):
+    """A listed position outside the block table's range sets MLA_ERR_BAD_BLOCK_ID and reads as a
+    zero row; the other sequences are unaffected."""
+    torch = _torch()
+    inp = small
+    rng = np.random.default_rng(5)
+    k = 64
+    idx = np.stack([np.sort(rng.choice(int(L), size=k, replace=False)) for L in inp["seq_lens"]]).astype(np.int32)
+    cnt = np.full(3, k, np.int32)
+    bad = idx.copy()
+    bad[1, 10] = inp["block_table"].shape[1] * 64 + 3
+    mla = _mla()
+    w = inp["workload"]
+    t = W.to_torch(inp)
+    out, lse = mla.sparse_decode(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], _dev(bad), _dev(cnt),
+                                 w.scale)
+    torch.cuda.synchronize()
+    assert mla.device_status() == 6
+    o, l = out.double().cpu().numpy(), lse.double().cpu().numpy()
+    assert np.isfinite(o).all() and np.isfinite(l).all()
+    ro, rl = oracle_sparse(inp, idx, cnt)
+    keep = [0, 2]
+    compare(o[keep], l[keep], ro[keep], rl[keep], TOL[W.BF16], "sequences without the bad position")
