@@ -330,7 +330,9 @@ mla_status_t mla_dsa_topk(const mla_dsa_params_t* params, const float* scores, c
 
 /* The decode's params (q_len 1, causal 0, BF16 cache, kernel AUTO or TCGEN05) and
  * workspace (mla_decode_workspace_size of the same params). indices [B, top_k] int32,
- * counts [B] int32, device. */
+ * counts [B] int32, device; 0 <= counts[b] <= top_k is the caller's to guarantee (the kernel
+ * reads indices[b, 0 .. counts[b]) and checks each position against the block table, not the
+ * count against top_k; mla_dsa_topk's outputs satisfy it). */
 mla_status_t mla_sparse_decode(const mla_decode_params_t* params, int32_t top_k, const void* q_lat,
                                const void* q_rope, const void* kv_cache, const int32_t* block_table,
                                const int32_t* indices, const int32_t* counts, void* out, float* lse,
