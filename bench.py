@@ -46,11 +46,15 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="deepseek_v3", choices=list(W.BY_NAME))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tcgen05"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tcgen05", "tc_pair"])
     ap.add_argument("--num-workers", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--extra-cpu-seconds", type=float, default=6.0,
+                    help="oracle sample per extra workload (the headline one gets --cpu-seconds)")
+    ap.add_argument("--only", action="store_true",
+                    help="time the chosen workload alone (by default one-GPU runs also time the other four)")
     ap.add_argument("--op", default="decode", choices=["decode", "append", "absorb", "project", "dsa"],
                     help="decode: the decode step (default); append: the paged cache append of the step's new "
                          "tokens; absorb / project: the per-head W^UK / W^UV products around the decode; dsa: "
@@ -78,7 +82,7 @@ MEASURED_TRAFFIC = {
     "524335d759a92050": {"deepseek_v3": (304.125184e6 + 4.850944e6) / 262144,
                          "fp8_cache": (169.770496e6 + 5.082368e6) / 262144},
 }
-KERNEL_SOURCES = ("mla_tc.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.h", "mla_tc.h")
+KERNEL_SOURCES = ("mla_pair.cu", "mla_tc.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.h", "mla_tc.h")
 # The same for the sparse step's indexer (dram bytes per context token, batch 8 of the
 # 128K workload), keyed by the sources of mla_dsa.cu and its headers.
 DSA_TRAFFIC = {
@@ -121,7 +125,9 @@ def job_rate_tbs(world: int, steps: int, bytes_per_step: float, max_ms: float) -
 
 
 def work_model(inp):
-    """Algorithmic bytes and FLOPs of one step ('Algorithmic work')."""
+    """Algorithmic bytes and FLOPs of one step: each attended cache token read once (1152 B bf16,
+    644 B e4m3 + bf16 RoPE key + fp32 scale), the queries read and the outputs written once;
+    2 (r + d_r) + 2 r FLOP per attended (query row, head, token)."""
     w = inp["workload"]
     lens = inp["seq_lens"].astype(np.int64)
     tok = int(lens.sum())
@@ -517,11 +523,45 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local))
 
-    import head_latent_attention_split_b200 as mla
     wl = W.BY_NAME[args.workload]
     if args.batch is not None and args.batch != wl.B:
         lens = wl.seq_lens if isinstance(wl.seq_lens, str) else tuple(wl.seq_lens[:1]) * args.batch
         wl = wl.with_(B=args.batch, seq_lens=lens, name=f"{wl.name}_b{args.batch}")
+    E = args.e2e_steps if args.e2e_steps is not None else max(1, min(args.steps, 50))
+    head = decode_workload(args, wl, world, rank, local, E, args.cpu_seconds)
+    # the other workloads of the pages (one GPU only: the scaling runs time the headline alone)
+    extra = {}
+    if world == 1 and not args.only and args.batch is None:
+        for other in W.WORKLOADS[1:]:
+            if other.name != wl.name:
+                extra[other.name] = decode_workload(args, other, world, rank, local, 0, args.extra_cpu_seconds)
+
+    if rank == 0:
+        r = head
+        line = dict(
+            metric=METRIC, value=r["value"], unit="TB/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+            ms_per_step=r["ms_per_step"], higher_is_better=True, scaling="weak", vs_baseline=None,
+            dtype=r["dtype"], data="synthetic", config=r["config"], tflops=r["tflops"], steps_per_s=r["steps_per_s"],
+            tokens_per_s=r["tokens_per_s"], step_ms_stats=r["step_ms_stats"], roofline=r["roofline"],
+            roofline_detail=r["roofline_detail"], cpu_baseline=r["cpu_baseline"], e2e=r["e2e"],
+            gpu_launches=2 * args.steps, clocks=r["clocks"])
+        if extra:
+            line["workloads"] = {name: {k: v for k, v in x.items() if k not in ("e2e", "value")} | {"tb_s": x["value"]}
+                                 for name, x in extra.items()}
+            line["gpu_launches"] += 2 * args.steps * len(extra)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def decode_workload(args, wl, world, rank, local, E, cpu_seconds):
+    """Time K decode steps of workload `wl` (CUDA events from mla_decode_timed on the launching
+    stream, max over ranks), then E end-to-end steps through mla_decode_host_io, then the oracle
+    on a bounded sample. Returns the figures of the JSON line for this workload."""
+    import torch
+    import torch.distributed as dist
+    import head_latent_attention_split_b200 as mla
     inp = W.make_inputs(wl, threads=max(1, (os.cpu_count() or 1) // world))
     t = W.to_torch(inp, f"cuda:{local}")
     p = mla.params_for(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], wl.scale, wl.causal,
@@ -553,7 +593,7 @@ def main():
     torch.cuda.synchronize()
     st = mla.device_status()
     if st != 0:
-        raise RuntimeError(f"device status {mla.status_string(st)}")
+        raise RuntimeError(f"{wl.name}: device status {mla.status_string(st)}")
 
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
@@ -583,83 +623,76 @@ def main():
     total_ms = reduce_max(sum(step_ms), world, out.device)
     st = mla.device_status()
     if st != 0:
-        raise RuntimeError(f"device status {mla.status_string(st)}")
+        raise RuntimeError(f"{wl.name}: device status {mla.status_string(st)}")
 
     # end-to-end through the host-buffer entry point: per-step inputs copied from pinned
     # host memory, result copied back, all inside the timed region
-    E = args.e2e_steps if args.e2e_steps is not None else max(1, min(K, 50))
-    pin = lambda x: x.cpu().pin_memory()
-    hq, hqr, hbt, hsl = pin(t["q_lat"]), pin(t["q_rope"]), pin(t["block_table"]), pin(t["seq_lens"])
-    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    hlse = torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
-    hws = torch.empty(mla.host_io_workspace_size(p), dtype=torch.uint8, device=out.device)
-    h2d = sum(x.numel() * x.element_size() for x in (hq, hqr, hbt, hsl))
-    d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
-    e2e_ms = 0.0
-    for i in range(E + 2 if E > 0 else 0):
-        if flush:
-            flush_buf.fill_(1.0)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        mla.mla_decode_host_io(p, hq, hqr, t["kv_cache"], t["k_rope_cache"], t["kv_scale"], hbt, hsl, hout, hlse,
-                               hws)
-        b.record()
-        b.synchronize()
-        if i >= 2:
-            e2e_ms += a.elapsed_time(b)
-    e2e_ms = reduce_max(e2e_ms, world, out.device)
+    e2e = None
+    if E > 0:
+        pin = lambda x: x.cpu().pin_memory()  # noqa: E731
+        hq, hqr, hbt, hsl = pin(t["q_lat"]), pin(t["q_rope"]), pin(t["block_table"]), pin(t["seq_lens"])
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        hlse = torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
+        hws = torch.empty(mla.host_io_workspace_size(p), dtype=torch.uint8, device=out.device)
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hqr, hbt, hsl))
+        d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
+        e2e_ms = 0.0
+        for i in range(E + 2):
+            if flush:
+                flush_buf.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            mla.mla_decode_host_io(p, hq, hqr, t["kv_cache"], t["k_rope_cache"], t["kv_scale"], hbt, hsl, hout, hlse,
+                                   hws)
+            b.record()
+            b.synchronize()
+            if i >= 2:
+                e2e_ms += a.elapsed_time(b)
+        e2e_ms = reduce_max(e2e_ms, world, out.device)
+        e2e = dict(value=job_rate_tbs(world, E, model["cache_bytes"], e2e_ms), unit="TB/s", h2d_bytes_per_step=h2d,
+                   d2h_bytes_per_step=d2h, ms_per_step=e2e_ms / E)
+        del hws
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu, _ = cpu_oracle_rate(inp, args.cpu_seconds)
+        cpu, _ = cpu_oracle_rate(inp, cpu_seconds)
+    del t, ws, out, lse, flush_buf
+    torch.cuda.empty_cache()
 
-    if rank == 0:
-        peaks = load_peaks()
-        sec = total_ms / 1e3
-        value = job_rate_tbs(world, K, model["cache_bytes"], total_ms)
-        dec_s = statistics.mean(dec_ms) / 1e3
-        t_hbm = model["bytes"] / (peaks["hbm_gbs"] * 1e9)
-        t_tc = model["flops"] / (peaks["bf16_tflops"] * 1e12)
-        bound = "hbm" if t_hbm >= t_tc else "tensor"
-        if bound == "hbm":
-            achieved, peak, unit = model["bytes"] / dec_s / 1e9, peaks["hbm_gbs"], "GB/s"
-        else:
-            achieved, peak, unit = model["flops"] / dec_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-        line = dict(
-            metric=METRIC, value=value, unit="TB/s", n_gpus=world, steps=K, warmup=args.warmup,
-            ms_per_step=total_ms / K, higher_is_better=True, scaling="weak", vs_baseline=None,
-            dtype=W.DTYPE_NAMES[wl.cache_dtype] if wl.cache_dtype != W.E4M3 else "e4m3+bf16",
-            data="synthetic",
-            config=dict(workload=wl.name, B=wl.B, Sq=wl.Sq, H=wl.H, r=wl.r, d_r=wl.d_r, block_size=wl.block_size,
-                        context=str(wl.seq_lens) if isinstance(wl.seq_lens, str) else int(max(wl.seq_lens)),
-                        cache=W.DTYPE_NAMES[wl.cache_dtype], kernel=kernel, workers=workers,
-                        parallelism=f"replicas x{world}" if world > 1 else "single GPU",
-                        l2=("flushed between steps (2x L2 buffer write)" if flush else
-                            f"inputs larger than L2 ({model['cache_bytes'] / 1e9:.2f} GB cache per step)"),
-                        resident_bytes=resident),
-            tflops=world * K * model["flops"] / sec / 1e12,
-            steps_per_s=K / sec,
-            tokens_per_s=world * K * wl.B * wl.Sq / sec,
-            roofline=dict(bound=bound, achieved=achieved, peak=peak, unit=unit, frac=achieved / peak,
-                          traffic=measured_traffic(wl, model, kernel)),
-            roofline_detail=dict(
-                kernel=f"decode ({kernel})", decode_ms=1e3 * dec_s, combine_ms=statistics.mean(comb_ms),
-                algorithmic_bytes=model["bytes"], algorithmic_flops=model["flops"],
-                hbm_gbs_achieved=model["bytes"] / dec_s / 1e9, tflops_achieved=model["flops"] / dec_s / 1e12,
-                hbm_frac=model["bytes"] / dec_s / 1e9 / peaks["hbm_gbs"],
-                tensor_frac=model["flops"] / dec_s / 1e12 / peaks["bf16_tflops"],
-                roofline_us=1e6 * max(t_hbm, t_tc), step_frac=max(t_hbm, t_tc) / (total_ms / K / 1e3),
-                peaks=peaks),
-            cpu_baseline=cpu,
-            e2e=dict(value=job_rate_tbs(world, E, model["cache_bytes"], e2e_ms), unit="TB/s",
-                     h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, ms_per_step=e2e_ms / E) if E > 0 else None,
-            gpu_launches=2 * K,
-            clocks=clocks,
-        )
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    peaks = load_peaks()
+    sec = total_ms / 1e3
+    dec_s = statistics.mean(dec_ms) / 1e3
+    t_hbm = model["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = model["flops"] / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    if bound == "hbm":
+        achieved, peak, unit = model["bytes"] / dec_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = model["flops"] / dec_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    stats = lambda xs: dict(mean=statistics.mean(xs), median=statistics.median(xs), min=min(xs))  # noqa: E731
+    return dict(
+        value=job_rate_tbs(world, K, model["cache_bytes"], total_ms), ms_per_step=total_ms / K,
+        dtype=W.DTYPE_NAMES[wl.cache_dtype] if wl.cache_dtype != W.E4M3 else "e4m3+bf16",
+        config=dict(workload=wl.name, B=wl.B, Sq=wl.Sq, H=wl.H, r=wl.r, d_r=wl.d_r, block_size=wl.block_size,
+                    context=str(wl.seq_lens) if isinstance(wl.seq_lens, str) else int(max(wl.seq_lens)),
+                    cache=W.DTYPE_NAMES[wl.cache_dtype], kernel=kernel, workers=workers,
+                    parallelism=f"replicas x{world}" if world > 1 else "single GPU",
+                    l2=("flushed between steps (2x L2 buffer write)" if flush else
+                        f"inputs larger than L2 ({model['cache_bytes'] / 1e9:.2f} GB cache per step)"),
+                    resident_bytes=resident),
+        tflops=world * K * model["flops"] / sec / 1e12, steps_per_s=K / sec, tokens_per_s=world * K * wl.B * wl.Sq / sec,
+        step_ms_stats=dict(step=stats(step_ms), decode=stats(dec_ms), combine=stats(comb_ms)),
+        roofline=dict(bound=bound, achieved=achieved, peak=peak, unit=unit, frac=achieved / peak,
+                      traffic=measured_traffic(wl, model, kernel)),
+        roofline_detail=dict(
+            kernel=f"decode ({kernel})", decode_ms=1e3 * dec_s, combine_ms=statistics.mean(comb_ms),
+            algorithmic_bytes=model["bytes"], algorithmic_flops=model["flops"],
+            hbm_gbs_achieved=model["bytes"] / dec_s / 1e9, tflops_achieved=model["flops"] / dec_s / 1e12,
+            hbm_frac=model["bytes"] / dec_s / 1e9 / peaks["hbm_gbs"],
+            tensor_frac=model["flops"] / dec_s / 1e12 / peaks["bf16_tflops"],
+            roofline_us=1e6 * max(t_hbm, t_tc), step_frac=max(t_hbm, t_tc) / (total_ms / K / 1e3),
+            peaks=peaks),
+        cpu_baseline=cpu, e2e=e2e, clocks=clocks)
 
 
 if __name__ == "__main__":

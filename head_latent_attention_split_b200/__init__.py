@@ -12,6 +12,6 @@ from .binding import (BF16, E4M3, F32, KERNELS, AppendParams, MlaError, Params, 
                       host_io_workspace_size, make_params, mla_decode, mla_decode_host_io, mla_decode_timed, plan_host,
                       mla_decode_noalloc, noalloc_max_workspace, DsaParams, make_dsa_params, mla_dsa_index,
                       mla_dsa_topk, mla_sparse_decode,
-                      plan_probe, resolve, status_string, workspace_size)
+                      plan_probe, resolve, set_wait_timeout_ns, status_string, wait_timeout_ns, workspace_size)
 from .api import (cache_append, decode, decode_host_io, dsa_index, dsa_params_for, dsa_topk,  # noqa: F401
                   head_gemm, params_for, sparse_decode)

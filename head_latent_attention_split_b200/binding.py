@@ -15,7 +15,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmla_decode.so")
 
 F32, BF16, E4M3 = 0, 1, 2
-KERNELS = {"auto": 0, "simt": 1, "tcgen05": 2}
+KERNELS = {"auto": 0, "simt": 1, "tcgen05": 2, "tc_pair": 3}
 KERNEL_NAMES = {v: k for k, v in KERNELS.items()}
 
 MLA_OK = 0
@@ -27,7 +27,7 @@ EXPORTED = ("mla_decode_workspace_size", "mla_decode_resolve", "mla_decode", "ml
             "mla_decode_host_io_workspace_size", "mla_decode_host_io", "mla_plan_host", "mla_plan_probe",
             "mla_get_device_status", "mla_status_string", "mla_abi_version", "mla_decode_noalloc",
             "mla_decode_noalloc_max_workspace", "mla_cache_append", "mla_head_gemm", "mla_dsa_index",
-            "mla_dsa_topk", "mla_sparse_decode")
+            "mla_dsa_topk", "mla_sparse_decode", "mla_set_wait_timeout_ns", "mla_get_wait_timeout_ns")
 
 
 class MlaError(RuntimeError):
@@ -95,6 +95,8 @@ def _load():
     L.mla_dsa_index.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.mla_dsa_topk.argtypes = [D, vp, vp, vp, vp, vp]
     L.mla_sparse_decode.argtypes = [P, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.mla_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+    L.mla_get_wait_timeout_ns.argtypes = []
     for name in EXPORTED:
         if not hasattr(L, name):
             raise ImportError(f"{LIB_PATH} lacks {name}: rebuild it")
@@ -102,6 +104,7 @@ def _load():
         if f.restype is ctypes.c_int and name != "mla_decode_noalloc_max_workspace":   # default
             f.restype = ctypes.c_int32
     L.mla_status_string.restype = ctypes.c_char_p
+    L.mla_get_wait_timeout_ns.restype = ctypes.c_uint64
     return L
 
 
@@ -254,6 +257,15 @@ def plan_probe(p: Params, block_table, seq_lens, stream=None):
     _check(lib.mla_plan_probe(ctypes.byref(p), _addr(block_table), _addr(seq_lens), _addr(slot), _addr(worker),
                               _addr(meta), _stream(stream)), "mla_plan_probe")
     return slot.view(p.batch, -1), worker.view(p.batch, -1), meta
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    """Limit of the kernels' bounded pipeline waits, process-wide (0 restores the 2 s default)."""
+    _check(lib.mla_set_wait_timeout_ns(int(ns)), "mla_set_wait_timeout_ns")
+
+
+def wait_timeout_ns() -> int:
+    return lib.mla_get_wait_timeout_ns()
 
 
 def status_string(st: int) -> str:

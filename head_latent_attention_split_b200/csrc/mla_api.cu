@@ -1,5 +1,6 @@
 // C-ABI host layer of libmla_decode.so: argument validation, kernel choice, workspace
 // layout, launches, the sticky device status word. See include/mla_decode.h.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -11,6 +12,8 @@
 namespace {
 
 __device__ int g_mla_status;   // sticky per-device status word (first error wins)
+
+std::atomic<uint64_t> g_wait_timeout_ns{mla::kDrainTimeoutNs};
 
 constexpr int kMaxDevices = 64;
 int* g_status_ptr[kMaxDevices];
@@ -59,7 +62,7 @@ mla_status_t check_shape(const mla_decode_params_t* p) {
   if (!triple_ok) return MLA_ERR_INVALID_ARG;
   if (!std::isfinite(p->softmax_scale)) return MLA_ERR_INVALID_ARG;
   if (p->causal != 0 && p->causal != 1) return MLA_ERR_INVALID_ARG;
-  if (p->kernel < MLA_KERNEL_AUTO || p->kernel > MLA_KERNEL_TCGEN05) return MLA_ERR_INVALID_ARG;
+  if (p->kernel < MLA_KERNEL_AUTO || p->kernel > MLA_KERNEL_TC_PAIR) return MLA_ERR_INVALID_ARG;
   // 32-bit token and slot indices inside the kernels
   if ((int64_t)p->max_blocks_per_seq * p->block_size > (1ll << 30)) return MLA_ERR_UNSUPPORTED;
   if ((int64_t)p->num_blocks * p->block_size > (1ll << 31) - 1) return MLA_ERR_UNSUPPORTED;
@@ -79,12 +82,13 @@ mla_status_t resolve(const mla_decode_params_t* p, int* kernel, int* workers) {
   int k = p->kernel;
   if (k == MLA_KERNEL_AUTO) k = (tc_ok && mla::kTcAuto) ? MLA_KERNEL_TCGEN05 : MLA_KERNEL_SIMT;
   if (k == MLA_KERNEL_TCGEN05 && !tc_ok) return MLA_ERR_UNSUPPORTED;
+  if (k == MLA_KERNEL_TC_PAIR && (!tc_ok || p->cache_dtype != MLA_DTYPE_BF16)) return MLA_ERR_UNSUPPORTED;
   if (k == MLA_KERNEL_SIMT && !simt_ok(p)) return MLA_ERR_UNSUPPORTED;
   int W = p->num_workers;
   if (W == 0) {
     const int sms = sm_count();
     if (sms <= 0) return MLA_ERR_CUDA;
-    if (k == MLA_KERNEL_TCGEN05) {
+    if (k == MLA_KERNEL_TCGEN05 || k == MLA_KERNEL_TC_PAIR) {
       W = mla::tc_auto_workers(sms, p->q_len * p->num_heads);
     } else {
       const int row_blocks = (p->q_len * p->num_heads + 7) / 8;
@@ -92,7 +96,7 @@ mla_status_t resolve(const mla_decode_params_t* p, int* kernel, int* workers) {
     }
     if (W < 1) W = 1;
   }
-  if (k == MLA_KERNEL_TCGEN05 && !mla::tc_workers_ok(W, p->q_len * p->num_heads)) return MLA_ERR_UNSUPPORTED;
+  if ((k == MLA_KERNEL_TCGEN05 || k == MLA_KERNEL_TC_PAIR) && !mla::tc_workers_ok(W, p->q_len * p->num_heads)) return MLA_ERR_UNSUPPORTED;
   if (W > 65535 * 8) return MLA_ERR_UNSUPPORTED;
   *kernel = k;
   *workers = W;
@@ -120,6 +124,7 @@ mla::DecodeArgs make_args(const mla_decode_params_t* p, int W) {
   a.out_dtype = p->out_dtype;
   a.causal = p->causal;
   a.rows = p->q_len * p->num_heads;
+  a.len_cap = p->max_blocks_per_seq * p->block_size;
   a.W = W;
   a.scale = p->softmax_scale;
   a.scale_log2 = (float)((double)p->softmax_scale * 1.4426950408889634);
@@ -128,9 +133,18 @@ mla::DecodeArgs make_args(const mla_decode_params_t* p, int W) {
 
 }  // namespace
 
+uint64_t mla::wait_timeout_ns() { return g_wait_timeout_ns.load(std::memory_order_relaxed); }
+
 extern "C" {
 
 int32_t mla_abi_version(void) { return MLA_DECODE_ABI_VERSION; }
+
+mla_status_t mla_set_wait_timeout_ns(uint64_t ns) {
+  g_wait_timeout_ns.store(ns ? ns : mla::kDrainTimeoutNs, std::memory_order_relaxed);
+  return MLA_OK;
+}
+
+uint64_t mla_get_wait_timeout_ns(void) { return mla::wait_timeout_ns(); }
 
 const char* mla_status_string(int32_t s) {
   switch (s) {
@@ -186,7 +200,7 @@ mla_status_t decode_impl(const mla_decode_params_t* p, const void* q_lat, const 
   if (workspace_bytes < L.total) return MLA_ERR_WORKSPACE_TOO_SMALL;
   if (!workspace) return MLA_ERR_INVALID_ARG;
   const void* ptrs[] = {q_lat, q_rope, kv_cache, k_rope_cache, kv_scale, block_table, seq_lens, out, lse};
-  const size_t need = kernel == MLA_KERNEL_TCGEN05 ? 16 : 4;
+  const size_t need = kernel == MLA_KERNEL_SIMT ? 4 : 16;
   for (const void* q : ptrs)
     if (q && !aligned(q, need)) return MLA_ERR_ALIGNMENT;
   if (!aligned(workspace, 256)) return MLA_ERR_ALIGNMENT;
@@ -214,7 +228,9 @@ mla_status_t decode_impl(const mla_decode_params_t* p, const void* q_lat, const 
     return !events || cudaEventRecord((cudaEvent_t)events[i], s) == cudaSuccess;
   };
   if (!record(0)) return MLA_ERR_CUDA;
-  cudaError_t e = kernel == MLA_KERNEL_TCGEN05 ? mla::launch_tc_decode(a, s) : mla::launch_simt_decode(a, s);
+  cudaError_t e = kernel == MLA_KERNEL_TCGEN05   ? mla::launch_tc_decode(a, s)
+                  : kernel == MLA_KERNEL_TC_PAIR ? mla::launch_pair_decode(a, s)
+                                                 : mla::launch_simt_decode(a, s);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (!record(1)) return MLA_ERR_CUDA;
   e = mla::launch_combine(a, s);
@@ -538,6 +554,7 @@ mla_status_t mla_sparse_decode(const mla_decode_params_t* p, int32_t top_k, cons
   a.seq_lens = counts;   // each sequence's length is its list's count
   a.sel_idx = indices;
   a.top_k = top_k;
+  if (top_k < a.len_cap) a.len_cap = top_k;   // a count above top_k is an error (and is clamped)
   a.out = out;
   a.lse = lse;
   char* ws = (char*)workspace;

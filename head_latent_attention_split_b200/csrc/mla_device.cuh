@@ -165,4 +165,29 @@ __device__ __forceinline__ int checked_block(const int32_t* __restrict__ bt, int
   return blk;
 }
 
+// Warp-collective: the part of sequence b in tiles [t0, t1) read something it may not: the
+// sequence's length is out of range, a block id is out of range, or (sparse decode, sel_idx set)
+// a listed position is outside the block table or maps to a bad block. Such rows are written as
+// NaN.
+__device__ __forceinline__ bool segment_poisoned(const DecodeArgs& a, int b, int t0, int t1) {
+  const int lane = threadIdx.x & 31;
+  const int L = __ldg(a.seq_lens + b);
+  bool bad = L < 0 || L > a.len_cap;
+  if (a.sel_idx == nullptr) {
+    for (int t = t0 + lane; t < t1; t += 32) {
+      const int blk = __ldg(a.block_table + (size_t)b * a.max_blocks + t);
+      bad |= blk < 0 || blk >= a.num_blocks;
+    }
+  } else if (!bad) {
+    const int pos_cap = a.max_blocks * a.bs;
+    const int j1 = min(t1 * a.bs, L);
+    for (int j = t0 * a.bs + lane; j < j1; j += 32) {
+      const int t = __ldg(a.sel_idx + (size_t)b * a.top_k + j);
+      const int blk = (t >= 0 && t < pos_cap) ? __ldg(a.block_table + (size_t)b * a.max_blocks + t / a.bs) : -1;
+      bad |= blk < 0 || blk >= a.num_blocks;
+    }
+  }
+  return __any_sync(0xffffffffu, bad);
+}
+
 }  // namespace mla

@@ -105,7 +105,8 @@ struct ItemWalk {
 
 __global__ void __launch_bounds__(kIThreads, kICtasPerSm)
     dsa_index_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_s, const DsaArgs a, const uint64_t timeout_ns) {
+                     const __grid_constant__ CUtensorMap tm_s, const DsaArgs a, const uint64_t timeout_ns,
+                     const uint64_t drain_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   IdxCtl& ctl = *reinterpret_cast<IdxCtl*>(smem + kIOffCtl);
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__(kIThreads, kICtasPerSm)
       // every load issued lands before the CTA may exit
       int dummy = 0;
       for (int i = max(0, issued - kIStages); i < issued; ++i)
-        mbar_wait<false>(smem_u32(&ctl.full[i % kIStages]), (i / kIStages) & 1, &dummy, timeout_ns);
+        mbar_wait<false>(smem_u32(&ctl.full[i % kIStages]), (i / kIStages) & 1, &dummy, drain_ns);
       if (!ok) {
         set_status(a.status, MLA_ERR_TIMEOUT);
         *abort = 1;
@@ -628,7 +629,7 @@ cudaError_t launch_dsa_index(const DsaArgs& a, cudaStream_t s) {
   // kICtasPerSm CTAs per SM, fewer when there are fewer tiles
   const long long tiles_max = (long long)R * ((a.max_seq_len + kITok - 1) / kITok);
   const int grid = (int)std::min<long long>((long long)kICtasPerSm * std::max(sms[dev & 63], 1), std::max(tiles_max, 1ll));
-  dsa_index_kernel<<<grid, kIThreads, kISmem, s>>>(tq, tk, ts, a, 2000000000ull);
+  dsa_index_kernel<<<grid, kIThreads, kISmem, s>>>(tq, tk, ts, a, wait_timeout_ns(), drain_timeout_ns());
   return cudaGetLastError();
 }
 

@@ -41,7 +41,7 @@ struct GemmCtl {
 template <int kNT>
 __global__ void __launch_bounds__(128, 1)
     head_gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                     const GemmArgs a, const uint64_t timeout_ns) {
+                     const GemmArgs a, const uint64_t timeout_ns, const uint64_t drain_ns) {
   constexpr uint32_t kStage = kAChunk + (kNT / 64) * kBChunk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -101,10 +101,10 @@ __global__ void __launch_bounds__(128, 1)
     }
     mma_commit(smem_u32(&ctl.done));
     int dummy = 0;
-    if (!mbar_wait<false>(smem_u32(&ctl.done), 0, &dummy, timeout_ns)) ok = false;
+    if (!mbar_wait<false>(smem_u32(&ctl.done), 0, &dummy, drain_ns)) ok = false;
     // loads still in flight land before the CTA may exit
     for (int kc = (nk > 2 ? nk - 2 : 0); kc < nk; ++kc)
-      mbar_wait<false>(smem_u32(&ctl.full[kc & 1]), (kc >> 1) & 1, &dummy, timeout_ns);
+      mbar_wait<false>(smem_u32(&ctl.full[kc & 1]), (kc >> 1) & 1, &dummy, drain_ns);
     if (!ok) {
       set_status(a.status, MLA_ERR_TIMEOUT);
       ctl.abort = 1;
@@ -190,7 +190,7 @@ cudaError_t launch_nt(const GemmArgs& a, cudaStream_t s) {
   });
   if (err != cudaSuccess) return err;
   const dim3 grid(a.n / kNT, a.heads, (a.rows + kGM - 1) / kGM);
-  head_gemm_kernel<kNT><<<grid, 128, smem, s>>>(tx, tw, a, 2000000000ull);
+  head_gemm_kernel<kNT><<<grid, 128, smem, s>>>(tx, tw, a, wait_timeout_ns(), drain_timeout_ns());
   return cudaGetLastError();
 }
 

@@ -20,6 +20,7 @@ struct DecodeArgs {
   int q_dtype, cache_dtype, out_dtype;
   int causal;
   int rows;            // Sq * H query rows per sequence
+  int len_cap;         // largest valid seq_lens entry: max_blocks * bs (sparse decode: also <= top_k)
   int W;               // workers sharing the flat block list
   float scale;         // softmax scale
   float scale_log2;    // softmax scale * log2(e)
@@ -48,6 +49,17 @@ struct WorkspaceLayout {
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Limit, in nanoseconds, of the bounded waits on a kernel's pipeline (default 2 s; set with
+// mla_set_wait_timeout_ns). A wait that runs out sets MLA_ERR_TIMEOUT.
+uint64_t wait_timeout_ns();
+// Limit of the waits that let a CTA's in-flight copies and MMAs land before it exits; never
+// shorter than the pipeline limit, so work already issued always completes.
+constexpr uint64_t kDrainTimeoutNs = 2000000000ull;
+inline uint64_t drain_timeout_ns() {
+  const uint64_t t = wait_timeout_ns();
+  return t > kDrainTimeoutNs ? t : kDrainTimeoutNs;
+}
 
 inline WorkspaceLayout workspace_layout(int B, int W, int rows, int r) {
   WorkspaceLayout L;

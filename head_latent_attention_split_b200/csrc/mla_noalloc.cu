@@ -11,10 +11,12 @@
 // Host code cannot use the array's name as a device address (it is a host-side stand-in),
 // so the first call on each device, with that device current, looks the address up with
 // cudaGetSymbolAddress and keeps it. Make that first call before any stream capture.
-// All calls on a device share the array and its contents persist between calls; the
-// decode writes every workspace word it later reads, so nothing needs clearing. Calls
-// whose work overlaps on the GPU (different streams, or host threads racing) race on the
-// array: serialise them.
+// All calls on a device share the array and its contents persist between calls. Nothing needs
+// clearing: the combine step recomputes each sequence's split from seq_lens and reads only the
+// partial slots that the decode kernel of the same call writes (with NaN when a wait ran out),
+// so a previous call's leftovers are never read. Calls whose work overlaps on the GPU
+// (different streams, or host threads racing) race on the array: serialise them.
+#include <atomic>
 #include <mutex>
 
 #include "../../include/mla_decode.h"
@@ -26,19 +28,19 @@ constexpr size_t kNoAllocScratchBytes = (size_t)MLA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_mla_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
-std::once_flag g_scratch_once[kMaxDevices];
+std::atomic<void*> g_scratch_ptr[kMaxDevices];
+std::mutex g_scratch_mu;
 
-// Device address of this device's scratch array (set-up on first use per device).
+// Device address of this device's scratch array, looked up on first use per device (with that
+// device current). A failed lookup is not remembered: the next call tries again.
 void* scratch_for(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::call_once(g_scratch_once[dev], [dev] {
-    void* p = nullptr;
-    g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_mla_scratch);
-    g_scratch_ptr[dev] = g_scratch_err[dev] == cudaSuccess ? p : nullptr;
-  });
-  return g_scratch_ptr[dev];
+  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
+  if (!p && cudaGetSymbolAddress(&p, g_mla_scratch) == cudaSuccess) g_scratch_ptr[dev].store(p, std::memory_order_release);
+  return g_scratch_ptr[dev].load(std::memory_order_relaxed);
 }
 
 }  // namespace

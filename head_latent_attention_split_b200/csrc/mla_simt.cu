@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kThreads) simt_decode_kernel(const DecodeArgs 
   const int row = blockIdx.y * kWarps + warp;
   const bool row_ok = row < a.rows;
   const int s = row_ok ? row / a.H : 0;
-  const int cap = a.max_blocks * a.bs;
+  const int cap = a.len_cap;
 
   if (warp == 0) {
     WorkerPlan p = warp_plan(a.seq_lens, a.B, a.bs, cap, a.W, w, a.status);
@@ -134,9 +134,11 @@ __global__ void __launch_bounds__(kThreads) simt_decode_kernel(const DecodeArgs 
         m = m_new;
       }
     }
+    const bool poisoned = segment_poisoned(a, b, sg.tile_begin, sg.tile_end);
     if (!row_ok) continue;
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    const float lse_v = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    const float qnan = __uint_as_float(0x7FC00000u);
+    const float inv = poisoned ? qnan : l > 0.f ? 1.f / l : 0.f;
+    const float lse_v = poisoned ? qnan : l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
     if (sg.splits == 1) {
 #pragma unroll
       for (int i = 0; i < kAV; ++i) {
@@ -156,27 +158,75 @@ __global__ void __launch_bounds__(kThreads) simt_decode_kernel(const DecodeArgs 
   }
 }
 
-// One warp per (b, row): merge the partials of split sequences, fill empty ones.
+// One warp per (b, row): merge the partials of split sequences, fill empty ones. The split of
+// each sequence is recomputed here from seq_lens with the plan's formula (nothing read from the
+// workspace is trusted for indexing). Rows of a sequence with a seq_len out of range, and rows
+// whose partials carry a NaN log-sum-exp (a decode wait timed out, or a bad block id), are
+// written as NaN.
 __global__ void __launch_bounds__(kThreads) combine_kernel(const DecodeArgs a) {
+  __shared__ long long s_sum[kWarps][2];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int b = blockIdx.x;
+  const int cap = a.len_cap;
+  // tiles before sequence b and in total, as the decode kernels' plan counts them
+  long long before = 0, total = 0;
+  for (int i = threadIdx.x; i < a.B; i += kThreads) {
+    const int L = __ldg(a.seq_lens + i);
+    const long long n = tiles_of(L < 0 ? 0 : (L > cap ? cap : L), a.bs);
+    total += n;
+    if (i < b) before += n;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+    total += __shfl_xor_sync(0xffffffffu, total, o);
+  }
+  if (lane == 0) {
+    s_sum[warp][0] = before;
+    s_sum[warp][1] = total;
+  }
+  __syncthreads();
+  before = total = 0;
+#pragma unroll
+  for (int i = 0; i < kWarps; ++i) {
+    before += s_sum[i][0];
+    total += s_sum[i][1];
+  }
   const int row = blockIdx.y * kWarps + warp;
   if (row >= a.rows) return;
-  const int cap = a.max_blocks * a.bs;
-  const int Lc = clamp_len(__ldg(a.seq_lens + b), cap, a.status);
   const size_t orow = (size_t)b * a.rows + row;
-  if (tiles_of(Lc, a.bs) == 0) {
+  const int raw = __ldg(a.seq_lens + b);
+  const float qnan = __uint_as_float(0x7FC00000u);
+  if (raw < 0 || raw > cap) {
+    for (int k = lane; k < a.r; k += 32) store_out(a.out, a.out_dtype, orow * a.r + k, qnan);
+    if (lane == 0) a.lse[orow] = qnan;
+    return;
+  }
+  const long long n = tiles_of(raw, a.bs);
+  if (n == 0) {
     for (int k = lane; k < a.r; k += 32) store_out(a.out, a.out_dtype, orow * a.r + k, 0.f);
     if (lane == 0) a.lse[orow] = -INFINITY;
     return;
   }
-  const int first = a.meta[2 * b], splits = a.meta[2 * b + 1];
-  if (splits <= 1) return;
+  const int Wa = (total < a.W) ? (int)total : a.W;
+  const int first = worker_of_tile(before, total, Wa);
+  const int splits = worker_of_tile(before + n - 1, total, Wa) - first + 1;
+  if (splits <= 1) return;   // the decode wrote this row directly
   const size_t slot0 = (size_t)first + b;
   float M = -INFINITY;
-  for (int i = lane; i < splits; i += 32) M = fmaxf(M, a.lse_part[(slot0 + i) * a.rows + row]);
+  bool has_nan = false;
+  for (int i = lane; i < splits; i += 32) {
+    const float v = a.lse_part[(slot0 + i) * a.rows + row];
+    has_nan |= v != v;
+    M = fmaxf(M, v);
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (__any_sync(0xffffffffu, has_nan)) {
+    for (int k = lane; k < a.r; k += 32) store_out(a.out, a.out_dtype, orow * a.r + k, qnan);
+    if (lane == 0) a.lse[orow] = qnan;
+    return;
+  }
   if (M == -INFINITY) {
     for (int k = lane; k < a.r; k += 32) store_out(a.out, a.out_dtype, orow * a.r + k, 0.f);
     if (lane == 0) a.lse[orow] = -INFINITY;
@@ -210,7 +260,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const DecodeArgs a) {
 __global__ void __launch_bounds__(32) plan_probe_kernel(const DecodeArgs a, int32_t* token_slot,
                                                          int32_t* token_worker) {
   const int w = blockIdx.x, lane = threadIdx.x;
-  const int cap = a.max_blocks * a.bs;
+  const int cap = a.len_cap;
   const WorkerPlan p = warp_plan(a.seq_lens, a.B, a.bs, cap, a.W, w, a.status);
   SegmentIter it(p, a.seq_lens, a.B, a.bs, cap, w, a.status);
   Segment sg;
@@ -222,7 +272,7 @@ __global__ void __launch_bounds__(32) plan_probe_kernel(const DecodeArgs a, int3
     const int t1 = min(sg.tile_end * a.bs, sg.Lc);
     for (int t = sg.tile_begin * a.bs + lane; t < t1; t += 32) {
       const int blk = checked_block(a.block_table, a.max_blocks, sg.b, t / a.bs, a.num_blocks, a.status);
-      const size_t o = (size_t)sg.b * cap + t;
+      const size_t o = (size_t)sg.b * a.max_blocks * a.bs + t;
       token_slot[o] = blk * a.bs + t % a.bs;
       token_worker[o] = w;
     }

@@ -129,6 +129,11 @@ constexpr uint32_t kFp8CodeBytes = kBS * 256;                    // this CTA's c
 constexpr uint32_t kFp8StageTx = kFp8CodeBytes + kKvRope + kBS * 4;   // codes, RoPE key, scales
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only if the max grows > 2^8
+// FP8 cache: the RoPE key is divided by max(s_t, 2^-64) and the score column multiplied by the
+// same factor. For s_t >= 2^-64 that is exact; below it (an all-zero latent stores s_t = 0, and
+// 1 / s_t would overflow for tiny scales) the latent term picks up an error of at most
+// 2^-64 * |q . code|, far below any tolerance, instead of inf * 0 = NaN.
+constexpr float kScaleFloor = 0x1p-64f;
 
 struct Ctl {
   uint64_t kv_full[kStages];
@@ -169,7 +174,7 @@ template <bool kFp8, bool kSparse>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(), 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_sc,
-                     const DecodeArgs a, const int n_rg, const uint64_t timeout_ns) {
+                     const DecodeArgs a, const int n_rg, const uint64_t timeout_ns, const uint64_t drain_ns) {
   using G = Geo<kFp8>;
   constexpr uint32_t kStageBytes = G::kStageBytes;
   constexpr uint32_t kOffKv = G::kOffKv;
@@ -183,7 +188,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
   const uint32_t peer = rank ^ 1u;
   const int cluster = (int)(blockIdx.x >> 1);
   const int w = cluster / n_rg, rg = cluster % n_rg;
-  const int cap = a.max_blocks * a.bs;
+  const int cap = a.len_cap;
   volatile int* abort = &ctl.abort;
 
   if (threadIdx.x == 0) {
@@ -263,7 +268,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
           int row = oob_row;
           if (j < sg.Lc) {
             const int t = __ldg(a.sel_idx + (size_t)sg.b * a.top_k + j);
-            const int blk = (t >= 0 && t < cap) ? __ldg(a.block_table + (size_t)sg.b * a.max_blocks + t / kBS) : -1;
+            const int blk = (t >= 0 && t < a.max_blocks * kBS) ? __ldg(a.block_table + (size_t)sg.b * a.max_blocks + t / kBS) : -1;
             if (blk >= 0 && blk < a.num_blocks)
               row = blk * kBS + t % kBS;
             else
@@ -299,7 +304,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
       int dummy = 0;
       for (uint32_t i = 0; i < kStages && i < g; ++i) {
         const uint32_t gl = g - 1 - i;
-        mbar_wait<false>(smem_u32(&ctl.kv_full[gl % kStages]), (gl / kStages) & 1, &dummy, timeout_ns);
+        mbar_wait<false>(smem_u32(&ctl.kv_full[gl % kStages]), (gl / kStages) & 1, &dummy, drain_ns);
       }
       if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
     }
@@ -341,7 +346,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
       int dummy = 0;
       for (uint32_t i = 0; i < kStages && i < g; ++i) {
         const uint32_t gl = g - 1 - i;   // the latest load of stage gl % kStages
-        mbar_wait<false>(smem_u32(&ctl.kv_full[gl % kStages]), (gl / kStages) & 1, &dummy, timeout_ns);
+        mbar_wait<false>(smem_u32(&ctl.kv_full[gl % kStages]), (gl / kStages) & 1, &dummy, drain_ns);
       }
       if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
     }
@@ -414,7 +419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
       // every MMA issued so far completes before TMEM can be released
       int dummy = 0;
       mma_commit(smem_u32(&ctl.drain));
-      mbar_wait<false>(smem_u32(&ctl.drain), 0, &dummy, timeout_ns);
+      mbar_wait<false>(smem_u32(&ctl.drain), 0, &dummy, drain_ns);
       if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
     }
   } else if (warp >= kConvWarp0) {
@@ -434,7 +439,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
           const float sc = *reinterpret_cast<const float*>(base + Geo<kFp8>::kOffScale + tok * 4);   // TMA'd
           // RoPE key / scale as bf16 hi + lo (its 64-byte row, 64B-swizzled, in place + lo slot)
           {
-            const float inv_sc = 1.0f / sc;
+            const float inv_sc = 1.0f / fmaxf(sc, kScaleFloor);
             uint8_t* hi_row = base + 4 * kKvLatChunk + tok * 64;
             uint8_t* lo_row = base + Geo<kFp8>::kOffRopeLo + tok * 64;
 #pragma unroll
@@ -573,7 +578,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
       mbar_arrive(smem_u32(&ctl.s_empty));
       return true;
     };
-    while (ok && it.next(sg)) {
+    while (it.next(sg)) {
+      bool written = false;   // this segment's rows of out / partials written
+      do {
+      if (!ok) break;
       // this segment's absorbed query, latent half of this CTA, into TMEM (the warp's 16 rows)
       ok = wait_local(smem_u32(&ctl.q_empty), (seg & 1) ^ 1);
       if (!ok) break;
@@ -619,8 +627,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
           const float4* cs = nullptr;   // FP8: token scales of my columns
           if constexpr (kFp8) {
             const uint32_t stg = gt % kStages;
-            int dummy = 0;
-            mbar_wait<false>(smem_u32(&ctl.kv_ready[stg]), (gt / kStages) & 1, &dummy, timeout_ns);
+            ok = wait_local(smem_u32(&ctl.kv_ready[stg]), (gt / kStages) & 1);
+            if (!ok) break;
             cs = reinterpret_cast<const float4*>(smem + kOffKv + stg * kStageBytes + G::kOffScale + 128 * hf);
           }
 #pragma unroll
@@ -634,10 +642,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
             float c4[4] = {1.f, 1.f, 1.f, 1.f};
             if constexpr (kFp8) {
               const float4 t = cs[c];
-              c4[0] = t.x;
-              c4[1] = t.y;
-              c4[2] = t.z;
-              c4[3] = t.w;
+              c4[0] = fmaxf(t.x, kScaleFloor);
+              c4[1] = fmaxf(t.y, kScaleFloor);
+              c4[2] = fmaxf(t.z, kScaleFloor);
+              c4[3] = fmaxf(t.w, kScaleFloor);
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -729,9 +737,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
           const int tail = sg.Lc % kBS;
           if (tile == last_tile && tail != 0) {
             const uint32_t stg = gt % kStages;
-            int dummy = 0;
-            mbar_wait<false>(smem_u32(kFp8 ? &ctl.kv_ready[stg] : &ctl.kv_full[stg]), (gt / kStages) & 1, &dummy,
-                             timeout_ns);
+            ok = wait_local(smem_u32(kFp8 ? &ctl.kv_ready[stg] : &ctl.kv_full[stg]), (gt / kStages) & 1);
+            if (!ok) break;
             uint8_t* base = smem + kOffKv + stg * kStageBytes;
             const int per_chunk = (kBS - tail) * 8;          // 16-byte pieces per chunk
             for (int i = threadIdx.x; i < 4 * per_chunk; i += 128) {   // the 4 own warps
@@ -851,7 +858,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
         __syncwarp();
         if (leader) mbar_arrive_expect_tx(smem_u32(&ctl.lrx_full[seg & 1]), kLrxBytes);   // segment seg + 2
       }
-      const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      const bool poisoned = segment_poisoned(a, sg.b, sg.tile_begin, sg.tile_end);
+      const float inv = poisoned ? __uint_as_float(0x7FC00000u) : l_tot > 0.f ? 1.f / l_tot : 0.f;
       const size_t qrow = (size_t)sg.b * a.rows + grow;
       const bool direct = sg.splits == 1;
       const size_t prow = (size_t)(w + sg.b) * a.rows + grow;
@@ -885,7 +893,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
         }
       }
       if (own && hf == 0 && valid_row) {
-        const float lse_v = l_tot > 0.f ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+        const float lse_v = poisoned ? __uint_as_float(0x7FC00000u)
+                            : l_tot > 0.f ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
         if (direct)
           a.lse[qrow] = lse_v;
         else
@@ -897,6 +906,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
       }
       tc_fence_before();
       ++seg;
+      written = true;
+      } while (0);
+      if (!written && valid_row) {
+        // a wait ran out: this CTA's channels of the segment's rows (and the lse) become NaN
+        const float qnan = __uint_as_float(0x7FC00000u);
+        const bool direct = sg.splits == 1;
+        const size_t qrow = (size_t)sg.b * a.rows + grow, prow = (size_t)(w + sg.b) * a.rows + grow;
+        for (int k = 0; k < 128; ++k) {
+          const int ch = 256 * (int)rank + 128 * hf + k;
+          if (direct && a.out_dtype == kBF16)
+            ((uint16_t*)a.out)[qrow * kR + ch] = 0x7FC0;
+          else
+            (direct ? (float*)a.out + qrow * kR : a.o_part + prow * kR)[ch] = qnan;
+        }
+        if (own && hf == 0) (direct ? a.lse[qrow] : a.lse_part[prow]) = qnan;
+      }
     }
     if (lane == 0) bulk_wait_group_read<0>();   // staging regions stay valid until read
     if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
@@ -1021,17 +1046,17 @@ cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, Geo<false>::kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  const uint64_t timeout_ns = 2000000000ull;
+  const uint64_t timeout_ns = wait_timeout_ns(), drain_ns = drain_timeout_ns();
   const dim3 grid(2 * a.W * n_rg);
   if (variant == 1)
     tc_decode_kernel<true, false><<<grid, threads_for<true>(), Geo<true>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a, n_rg,
-                                                                                           timeout_ns);
+                                                                                           timeout_ns, drain_ns);
   else if (variant == 2)
     tc_decode_kernel<false, true><<<grid, threads_for<false>(), Geo<false>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a,
-                                                                                             n_rg, timeout_ns);
+                                                                                             n_rg, timeout_ns, drain_ns);
   else
     tc_decode_kernel<false, false><<<grid, threads_for<false>(), Geo<false>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a,
-                                                                                              n_rg, timeout_ns);
+                                                                                              n_rg, timeout_ns, drain_ns);
   return cudaGetLastError();
 }
 

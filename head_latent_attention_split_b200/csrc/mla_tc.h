@@ -16,4 +16,7 @@ int tc_auto_workers(int sms, int rows);
 bool tc_workers_ok(int W, int rows);
 cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s);
 
+// Split-role pair kernel (mla_pair.cu): bf16 cache, dense token ranges.
+cudaError_t launch_pair_decode(const DecodeArgs& a, cudaStream_t s);
+
 }  // namespace mla

@@ -52,12 +52,15 @@
  *
  * Errors. Argument errors are detected on the host before anything is enqueued and
  * returned synchronously (nothing is launched). A failed launch returns MLA_ERR_CUDA.
- * Data-dependent errors found on the device (a block id outside [0, num_blocks), a
- * seq_len outside [0, max_blocks_per_seq * block_size], a bounded wait that timed
- * out) do not stop the kernels: the offending block id is replaced by block 0 and the
- * seq_len clamped, so the results for that sequence are meaningless, and a sticky
- * per-device status word records the first such error. mla_get_device_status() reads
- * and clears it. No device code traps.
+ * Data-dependent errors found on the device do not stop the other sequences of the
+ * call, and they are visible in the output: every row (out and lse) of a sequence whose
+ * seq_len is outside [0, max_blocks_per_seq * block_size], or whose block table names a
+ * block outside [0, num_blocks) within its length, is written as NaN; so is every row a
+ * kernel did not finish because one of its bounded waits ran out (see
+ * mla_set_wait_timeout_ns). A sticky per-device status word records the first such
+ * error (MLA_ERR_BAD_SEQ_LEN, MLA_ERR_BAD_BLOCK_ID, MLA_ERR_TIMEOUT);
+ * mla_get_device_status() reads and clears it. No device code traps, and the context
+ * stays usable.
  */
 #ifndef MLA_DECODE_H_
 #define MLA_DECODE_H_
@@ -88,7 +91,9 @@ typedef enum {
 typedef enum {
   MLA_KERNEL_AUTO = 0,     /* tensor-core kernel when the shape allows it, else SIMT */
   MLA_KERNEL_SIMT = 1,     /* fp32 CUDA-core kernel: any r <= 1024, r + d_r <= 1280 */
-  MLA_KERNEL_TCGEN05 = 2   /* tcgen05/TMA kernel: r = 512, d_r = 64, block_size = 64 */
+  MLA_KERNEL_TCGEN05 = 2,  /* tcgen05/TMA kernel: r = 512, d_r = 64, block_size = 64 */
+  MLA_KERNEL_TC_PAIR = 3   /* split-role tcgen05/TMA kernel on CTA pairs (scores on one CTA, P.V on its
+                              peer): the shapes of MLA_KERNEL_TCGEN05 with a bf16 cache; dense decode only */
 } mla_kernel_t;
 
 typedef struct {
@@ -199,6 +204,18 @@ mla_status_t mla_plan_probe(const mla_decode_params_t* params, const int32_t* bl
  * (MLA_OK or one of the device-detected codes). Returns MLA_ERR_CUDA if the
  * synchronisation itself failed. */
 mla_status_t mla_get_device_status(void* stream, int32_t* device_status);
+
+/* Limit, in nanoseconds, of every bounded wait inside the library's kernels (pipeline
+ * hand-offs between warps and between the CTAs of a cluster). Default 2e9 (2 s); 0
+ * restores the default. A wait that runs out ends its kernel's work early: the rows it
+ * did not finish are NaN and MLA_ERR_TIMEOUT is recorded in the status word. The waits
+ * that let already-issued copies and MMAs complete before a CTA exits keep a limit of at
+ * least 2 s, so a short limit never leaves work in flight. Process-wide; it applies to
+ * launches enqueued after the call (meant for tests and watchdogs). No counterpart in the
+ * papers: it is a property of this library's kernels. */
+mla_status_t mla_set_wait_timeout_ns(uint64_t ns);
+/* The limit currently in force. */
+uint64_t mla_get_wait_timeout_ns(void);
 
 /* Static, human-readable name of a status code. */
 const char* mla_status_string(int32_t status);

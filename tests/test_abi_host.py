@@ -105,6 +105,10 @@ def test_unsupported_kernel_requests(m):
     assert _call(m, _p(m, r=2048)) == 2
     # the tensor-core kernel needs r = 512, d_r = 64, block 64, bf16 queries
     assert _call(m, _p(m, kernel="tcgen05")) == 2
+    assert _call(m, _p(m, kernel="tc_pair")) == 2
+    # the pair kernel reads bf16 caches only
+    tc_shape = dict(r=512, d_r=64, block_size=64, q_dtype=1, cache_dtype=1, out_dtype=1)
+    assert _call(m, _p(m, kernel="tc_pair", **{**tc_shape, "cache_dtype": 2})) == 2
 
 
 def test_batch_zero_is_a_noop(m):
@@ -261,7 +265,7 @@ def _sparse(m, **kw):
 
 
 @pytest.mark.parametrize("bad,code", [(dict(Sq=2), 2), (dict(causal=True), 2), (dict(cache_dtype=2), 2),
-                                      (dict(kernel="simt"), 2), (dict(top_k=0), 1), (dict(indices=None), 1),
+                                      (dict(kernel="simt"), 2), (dict(kernel="tc_pair"), 2), (dict(top_k=0), 1), (dict(indices=None), 1),
                                       (dict(counts=None), 1), (dict(q_rope=None), 1), (dict(workspace_bytes=16), 4),
                                       (dict(q_lat=FAKE + 8), 3), (dict(indices=FAKE + 2), 3)])
 def test_sparse_decode_rejects_bad_arguments_on_host(m, bad, code):

@@ -371,8 +371,8 @@ def test_index_bad_block_id_and_seq_len_set_status(small):
 
 
 def test_sparse_decode_bad_position_sets_status(small):
-    """A listed position outside the block table's range sets MLA_ERR_BAD_BLOCK_ID and reads as a
-    zero row; the other sequences are unaffected."""
+    """A listed position outside the block table's range sets MLA_ERR_BAD_BLOCK_ID and turns that
+    sequence's rows NaN; the other sequences are unaffected."""
     torch = _torch()
     inp = small
     rng = np.random.default_rng(5)
@@ -389,7 +389,32 @@ def test_sparse_decode_bad_position_sets_status(small):
     torch.cuda.synchronize()
     assert mla.device_status() == 6
     o, l = out.double().cpu().numpy(), lse.double().cpu().numpy()
-    assert np.isfinite(o).all() and np.isfinite(l).all()
+    assert np.isnan(o[1]).all() and np.isnan(l[1]).all()
     ro, rl = oracle_sparse(inp, idx, cnt)
     keep = [0, 2]
     compare(o[keep], l[keep], ro[keep], rl[keep], TOL[W.BF16], "sequences without the bad position")
+
+
+def test_sparse_decode_count_above_top_k_sets_status(small):
+    """A count above top_k (the list's row stride) is an error: MLA_ERR_BAD_SEQ_LEN, that
+    sequence's rows NaN, nothing read past its list; the other sequences are unaffected."""
+    torch = _torch()
+    inp = small
+    rng = np.random.default_rng(6)
+    k = 64
+    idx = np.stack([np.sort(rng.choice(int(L), size=k, replace=False)) for L in inp["seq_lens"]]).astype(np.int32)
+    cnt = np.full(3, k, np.int32)
+    bad = cnt.copy()
+    bad[2] = k + 5          # the last row: a read past the count would run off the indices buffer
+    mla = _mla()
+    w = inp["workload"]
+    t = W.to_torch(inp)
+    out, lse = mla.sparse_decode(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], _dev(idx), _dev(bad),
+                                 w.scale)
+    torch.cuda.synchronize()
+    assert mla.device_status() == 7
+    o, l = out.double().cpu().numpy(), lse.double().cpu().numpy()
+    assert np.isnan(o[2]).all() and np.isnan(l[2]).all()
+    ro, rl = oracle_sparse(inp, idx, cnt)
+    keep = [0, 1]
+    compare(o[keep], l[keep], ro[keep], rl[keep], TOL[W.BF16], "sequences with a valid count")

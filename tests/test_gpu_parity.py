@@ -16,7 +16,7 @@ from parity_util import TOL, compare, run_gpu, sample_rows
 
 pytestmark = pytest.mark.gpu
 
-KERNELS = ["simt", "tcgen05"]
+KERNELS = ["simt", "tcgen05", "tc_pair"]
 
 
 @pytest.fixture(scope="module")
@@ -51,6 +51,13 @@ SMALL = {
     "mtp_causal_short": W.WORKLOADS[3].with_(B=3, seq_lens=(1, 0, 64)),
     "fp8": W.WORKLOADS[4].with_(B=4, seq_lens=(5, 64, 200, 1500)),
     "fp8_h32": W.WORKLOADS[4].with_(B=2, H=32, seq_lens=(129, 1000)),
+    # all-zero latents (scale 0, what the cache append stores for them) and tiny scales whose
+    # reciprocal overflows fp32 (2^-130 latents: scale ~2^-137, subnormal; 2^-120 latents)
+    "fp8_zero_tiny130": W.WORKLOADS[4].with_(B=3, seq_lens=(130, 700, 64), zero_every=7, tiny_every=11,
+                                             tiny_exp=-130),
+    "fp8_zero_tiny120": W.WORKLOADS[4].with_(B=2, seq_lens=(1000, 77), zero_every=3, tiny_every=5,
+                                             tiny_exp=-120),
+    "bf16_zero_tokens": W.WORKLOADS[2].with_(B=2, seq_lens=(200, 513), zero_every=5),
     "sharp_softmax": W.WORKLOADS[2].with_(B=2, seq_lens=(300, 513), scale=8.0 / math.sqrt(192.0)),
     "scale_zero": W.WORKLOADS[2].with_(B=2, seq_lens=(100, 257), scale=0.0),
 }
@@ -165,30 +172,81 @@ def test_plan_probe_bit_exact(mla):
         assert mla.device_status() == 0
 
 
+def _check_nan_rows(out, lse, bad, ref_o, ref_l, tol, what):
+    """Every row of the sequences in `bad` is NaN (out and lse); the others match the oracle."""
+    o = out.double().cpu().numpy()
+    l = lse.double().cpu().numpy()
+    good = [b for b in range(o.shape[0]) if b not in bad]
+    for b in bad:
+        assert np.isnan(o[b]).all() and np.isnan(l[b]).all(), f"{what}: sequence {b} not NaN"
+    compare(o[good], l[good], ref_o[good], ref_l[good], tol, what)
+
+
 @pytest.mark.parametrize("kernel", KERNELS)
-def test_bad_block_id_and_seq_len_set_status(mla, small_cases, kernel):
+@pytest.mark.parametrize("num_workers", [0, 1, 7])
+def test_bad_block_id_and_seq_len_set_status(mla, small_cases, kernel, num_workers):
+    """A bad block id or seq_len sets the sticky status and turns that sequence's rows NaN;
+    the other sequences still match the oracle (also when the bad one is split over workers)."""
     import torch
-    inp, _ = small_cases("bf16_h128")
-    if not kernel_ok(mla, inp, kernel):
+    inp, (ref_o, ref_l) = small_cases("bf16_h128")
+    if not kernel_ok(mla, inp, kernel, num_workers):
         pytest.skip(kernel)
     w = inp["workload"]
+    tol = TOL[w.cache_dtype]
     t = W.to_torch(inp)
-    bt = t["block_table"].clone()
-    bt[3, 2] = inp["num_blocks"] + 17
-    mla.decode(t["q_lat"], t["q_rope"], t["kv_cache"], bt, t["seq_lens"], w.scale, kernel=kernel)
-    assert mla.device_status() == 6           # MLA_ERR_BAD_BLOCK_ID
-    assert mla.device_status() == 0           # cleared by the read
+    args = dict(num_workers=num_workers, kernel=kernel)
+    for blk in (inp["num_blocks"] + 17, -1):
+        bt = t["block_table"].clone()
+        bt[3, 2] = blk
+        out, lse = mla.decode(t["q_lat"], t["q_rope"], t["kv_cache"], bt, t["seq_lens"], w.scale, **args)
+        torch.cuda.synchronize()
+        assert mla.device_status() == 6           # MLA_ERR_BAD_BLOCK_ID
+        assert mla.device_status() == 0           # cleared by the read
+        _check_nan_rows(out, lse, {3}, ref_o, ref_l, tol, f"bad block {blk}")
     sl = t["seq_lens"].clone()
-    sl[1] = inp["max_blocks_per_seq"] * 64 + 1
-    mla.decode(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], sl, w.scale, kernel=kernel)
-    assert mla.device_status() == 7           # MLA_ERR_BAD_SEQ_LEN
-    sl[1] = -5
-    mla.decode(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], sl, w.scale, kernel=kernel)
-    assert mla.device_status() == 7
+    for bad_len in (inp["max_blocks_per_seq"] * 64 + 1, -5):
+        sl[1] = bad_len
+        out, lse = mla.decode(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], sl, w.scale, **args)
+        torch.cuda.synchronize()
+        assert mla.device_status() == 7           # MLA_ERR_BAD_SEQ_LEN
+        _check_nan_rows(out, lse, {1}, ref_o, ref_l, tol, f"bad seq_len {bad_len}")
     # the stream and context stay usable: a clean call still matches
-    o, l = run_gpu(inp, kernel, 0, tensors=t)
-    assert np.isfinite(o).all()
-    torch.cuda.synchronize()
+    o, l = run_gpu(inp, kernel, num_workers, tensors=t)
+    compare(o, l, ref_o, ref_l, tol, "after the bad calls")
+
+
+def test_wait_timeout_expires_cleanly(mla, small_cases):
+    """A pipeline wait limit far below the time a tile takes makes the tensor-core kernel's
+    waits run out: the call returns, the status word reads MLA_ERR_TIMEOUT once, the unfinished
+    rows are NaN, and the next call with the default limit matches the oracle."""
+    import torch
+    inp, (ref_o, ref_l) = small_cases("bf16_h128")
+    if not kernel_ok(mla, inp, "tcgen05"):
+        pytest.skip("tcgen05")
+    w = inp["workload"]
+    t = W.to_torch(inp)
+    assert mla.wait_timeout_ns() == 2_000_000_000
+    mla.set_wait_timeout_ns(200)
+    try:
+        assert mla.wait_timeout_ns() == 200
+        out, lse = mla.decode(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], t["seq_lens"], w.scale,
+                              kernel="tcgen05")
+        torch.cuda.synchronize()
+    finally:
+        mla.set_wait_timeout_ns(0)
+    assert mla.wait_timeout_ns() == 2_000_000_000
+    assert mla.device_status() == 8           # MLA_ERR_TIMEOUT
+    assert mla.device_status() == 0
+    o = out.double().cpu().numpy()
+    l = lse.double().cpu().numpy()
+    assert np.isnan(o).any() and np.isnan(l).any()
+    # every row is either NaN throughout or the right answer
+    for b in range(w.B):
+        for h in range(w.H):
+            if np.isnan(l[b, 0, h]):
+                assert np.isnan(o[b, 0, h]).all()
+    o2, l2 = run_gpu(inp, "tcgen05", 0, tensors=t)
+    compare(o2, l2, ref_o, ref_l, TOL[w.cache_dtype], "after the timeout")
 
 
 @pytest.mark.parametrize("kernel", KERNELS)

@@ -4,9 +4,10 @@ mla_decode_noalloc exists for callers that may not allocate device memory while 
 decode: a serving engine that reserved the GPU's memory for its cache before the first
 step, or a plugin that runs in a memory pool it does not own. It takes the same inputs
 and outputs as mla_decode but no workspace; the split workspace is the library's own
-fixed-size device array. Two calls in a row must give what mla_decode gives (the array
-keeps the previous call's contents, so the second call checks that stale contents do
-not leak into the result).
+fixed-size device array. Calls in a row must each give what mla_decode gives: the array
+keeps the previous call's contents, so a large call (more sequences, more workers, more
+split partials) runs first and the smaller call after it checks that none of the larger
+call's leftovers leak into the result.
 """
 import numpy as np
 import pytest
@@ -25,25 +26,21 @@ def _mla():
     return mla
 
 
-@pytest.mark.gpu
-@pytest.mark.parametrize("wl", [W.WORKLOADS[3].with_(B=4, seq_lens=(2, 65, 300, 777)),
-                                W.WORKLOADS[4].with_(B=3, seq_lens=(5, 200, 1500))],
-                         ids=["bf16_causal", "fp8"])
-def test_noalloc_matches_workspace_entry_point(wl):
+def _noalloc_vs_workspace(mla, wl, num_workers, calls):
+    """Run mla_decode_noalloc `calls` times on workload wl and compare each result with
+    mla_decode's (same parameters, caller-owned workspace)."""
     import torch
-    mla = _mla()
     inp = W.make_inputs(wl)
     t = W.to_torch(inp)
-    # five workers split the longer sequences, so the scratch array carries partials
     p = mla.params_for(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], wl.scale, wl.causal,
-                       num_workers=5)
+                       num_workers=num_workers)
     assert mla.workspace_size(p) <= mla.noalloc_max_workspace()
     ref_o, ref_l = mla.decode(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], t["seq_lens"], wl.scale,
-                              wl.causal, t["k_rope_cache"], t["kv_scale"], num_workers=5)
+                              wl.causal, t["k_rope_cache"], t["kv_scale"], num_workers=num_workers)
     torch.cuda.synchronize()
     ref_o = ref_o.double().cpu().numpy()
     ref_l = ref_l.double().cpu().numpy()
-    for call in range(2):
+    for call in range(calls):
         out = torch.full(t["q_lat"].shape, float("nan"), dtype=torch.bfloat16, device="cuda")
         lse = torch.full(t["q_lat"].shape[:3], float("nan"), dtype=torch.float32, device="cuda")
         mla.mla_decode_noalloc(p, t["q_lat"], t["q_rope"], t["kv_cache"], t["k_rope_cache"], t["kv_scale"],
@@ -52,10 +49,23 @@ def test_noalloc_matches_workspace_entry_point(wl):
         assert mla.device_status() == 0
         o = out.double().cpu().numpy()
         l = lse.double().cpu().numpy()
-        assert np.isfinite(o).all(), f"call {call}: non-finite output"
+        assert np.isfinite(o).all(), f"{wl.name} call {call}: non-finite output"
         err = np.abs(o - ref_o).max() / np.abs(ref_o).max()
-        assert err <= TOL[wl.cache_dtype], f"call {call}: {err}"
-        assert np.abs(l - ref_l).max() <= LSE_TOL, f"call {call}: lse"
+        assert err <= TOL[wl.cache_dtype], f"{wl.name} call {call}: {err}"
+        assert np.abs(l - ref_l).max() <= LSE_TOL, f"{wl.name} call {call}: lse"
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl", [W.WORKLOADS[3].with_(B=4, seq_lens=(2, 65, 300, 777)),
+                                W.WORKLOADS[4].with_(B=3, seq_lens=(5, 200, 1500))],
+                         ids=["bf16_causal", "fp8"])
+def test_noalloc_matches_workspace_entry_point(wl):
+    mla = _mla()
+    # a larger call first (more sequences and workers: more split partials in the array) ...
+    big = wl.with_(B=12, seq_lens=tuple((list(W.resolve_seq_lens(wl)) * 4)[:12]))
+    _noalloc_vs_workspace(mla, big, 40, 1)
+    # ... then the small one twice: five workers split its longer sequences
+    _noalloc_vs_workspace(mla, wl, 5, 2)
 
 
 def test_noalloc_rejects_workspace_beyond_its_array():

@@ -58,6 +58,9 @@ class Workload:
     outlier_gain: float = 8.0
     contiguous: bool = False       # block_table = identity layout instead of a permutation
     spare_blocks: int = 0          # physical blocks owned by no sequence (poisoned)
+    zero_every: int = 0            # > 0: every zero_every-th cache slot (from slot 1) holds an all-zero latent
+    tiny_every: int = 0            # > 0: every tiny_every-th slot (from slot 2) has its latent scaled by 2^tiny_exp
+    tiny_exp: int = -130
     seed: int = 0
     block_size: int = BLOCK
     description: str = ""
@@ -152,12 +155,13 @@ def quantize_e4m3_per_token(c: np.ndarray):
     """Per-token e4m3 storage: scale = amax/448, code = RNE(c/scale) (OCP e4m3, no inf).
 
     Uses torch's float8_e4m3fn cast as the rounding routine. Tokens whose amax is 0
-    get scale 1 and all-zero codes.
+    get scale 0 and all-zero codes (what the library's cache append stores for them).
     """
     import torch
     amax = np.abs(c).max(axis=-1)
-    scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
-    y = np.clip(c / scale[..., None], -448.0, 448.0).astype(np.float32)
+    scale = (amax / np.float32(448.0)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    y = np.clip(c / safe[..., None], -448.0, 448.0).astype(np.float32)
     codes = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     return codes, scale
 
@@ -200,6 +204,11 @@ def make_inputs(w: Workload, threads: int | None = None) -> dict:
         n_out = max(1, int(round(w.outlier_frac * w.r)))
         ch = np.random.default_rng(np.random.SeedSequence([w.seed, 11])).choice(w.r, n_out, replace=False)
         c[:, :, np.sort(ch)] *= np.float32(w.outlier_gain)
+    flat = c.reshape(-1, w.r)
+    if w.zero_every > 0:
+        flat[1::w.zero_every] = 0.0
+    if w.tiny_every > 0:
+        flat[2::w.tiny_every] *= np.float32(2.0 ** w.tiny_exp)
 
     # slots no sequence may read: tokens past seq_len in each last block, spare blocks
     poison = np.zeros((num_blocks, bs), dtype=bool)
