@@ -74,13 +74,19 @@ bool simt_ok(const mla_decode_params_t* p) {
 }
 
 // Resolve the kernel and the worker count. needs_device: the SM count was required.
-mla_status_t resolve(const mla_decode_params_t* p, int* kernel, int* workers) {
+// sparse: the call is a sparse decode (AUTO then keeps the single-CTA tensor-core kernel).
+mla_status_t resolve(const mla_decode_params_t* p, int* kernel, int* workers, bool sparse = false) {
   mla_status_t st = check_shape(p);
   if (st) return st;
   const bool tc_ok = mla::tc_supported(p->kv_rank, p->rope_dim, p->block_size, p->q_dtype, p->cache_dtype,
                                        p->out_dtype, p->q_len * p->num_heads);
   int k = p->kernel;
-  if (k == MLA_KERNEL_AUTO) k = (tc_ok && mla::kTcAuto) ? MLA_KERNEL_TCGEN05 : MLA_KERNEL_SIMT;
+  if (k == MLA_KERNEL_AUTO) {
+    if (!tc_ok || !mla::kTcAuto)
+      k = MLA_KERNEL_SIMT;
+    else
+      k = (!sparse && p->cache_dtype == MLA_DTYPE_BF16) ? MLA_KERNEL_TC_PAIR : MLA_KERNEL_TCGEN05;
+  }
   if (k == MLA_KERNEL_TCGEN05 && !tc_ok) return MLA_ERR_UNSUPPORTED;
   if (k == MLA_KERNEL_TC_PAIR && (!tc_ok || p->cache_dtype != MLA_DTYPE_BF16)) return MLA_ERR_UNSUPPORTED;
   if (k == MLA_KERNEL_SIMT && !simt_ok(p)) return MLA_ERR_UNSUPPORTED;
@@ -529,7 +535,7 @@ mla_status_t mla_sparse_decode(const mla_decode_params_t* p, int32_t top_k, cons
                                const int32_t* indices, const int32_t* counts, void* out, float* lse,
                                void* workspace, size_t workspace_bytes, void* stream) {
   int kernel = 0, W = 0;
-  mla_status_t st = resolve(p, &kernel, &W);
+  mla_status_t st = resolve(p, &kernel, &W, true);
   if (st) return st;
   if (top_k < 1) return MLA_ERR_INVALID_ARG;
   if (p->q_len != 1 || p->causal != 0 || p->cache_dtype != MLA_DTYPE_BF16 || kernel != MLA_KERNEL_TCGEN05)

@@ -89,7 +89,8 @@ typedef enum {
 } mla_status_t;
 
 typedef enum {
-  MLA_KERNEL_AUTO = 0,     /* tensor-core kernel when the shape allows it, else SIMT */
+  MLA_KERNEL_AUTO = 0,     /* tensor-core kernel when the shape allows it (TC_PAIR for a bf16 cache,
+                              TCGEN05 for an FP8 cache and for sparse decode), else SIMT */
   MLA_KERNEL_SIMT = 1,     /* fp32 CUDA-core kernel: any r <= 1024, r + d_r <= 1280 */
   MLA_KERNEL_TCGEN05 = 2,  /* tcgen05/TMA kernel: r = 512, d_r = 64, block_size = 64 */
   MLA_KERNEL_TC_PAIR = 3   /* split-role tcgen05/TMA kernel on CTA pairs (scores on one CTA, P.V on its

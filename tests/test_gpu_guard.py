@@ -44,6 +44,8 @@ CASES = [
     ("tcgen05", W.WORKLOADS[2].with_(B=3, seq_lens=(1, 700, 129)), 0),
     ("tcgen05", W.WORKLOADS[3].with_(B=3, seq_lens=(2, 300, 65)), 500),
     ("tcgen05", W.WORKLOADS[4].with_(B=2, seq_lens=(64, 1100)), 1),
+    ("tc_pair", W.WORKLOADS[2].with_(B=3, seq_lens=(1, 700, 129)), 0),
+    ("tc_pair", W.WORKLOADS[3].with_(B=3, seq_lens=(2, 300, 65)), 500),
     ("simt", W.WORKLOADS[1].with_(B=2, seq_lens=(3, 200)), 7),
 ]
 

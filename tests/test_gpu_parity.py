@@ -215,14 +215,15 @@ def test_bad_block_id_and_seq_len_set_status(mla, small_cases, kernel, num_worke
     compare(o, l, ref_o, ref_l, tol, "after the bad calls")
 
 
-def test_wait_timeout_expires_cleanly(mla, small_cases):
+@pytest.mark.parametrize("kernel", ["tcgen05", "tc_pair"])
+def test_wait_timeout_expires_cleanly(mla, small_cases, kernel):
     """A pipeline wait limit far below the time a tile takes makes the tensor-core kernel's
     waits run out: the call returns, the status word reads MLA_ERR_TIMEOUT once, the unfinished
     rows are NaN, and the next call with the default limit matches the oracle."""
     import torch
     inp, (ref_o, ref_l) = small_cases("bf16_h128")
-    if not kernel_ok(mla, inp, "tcgen05"):
-        pytest.skip("tcgen05")
+    if not kernel_ok(mla, inp, kernel):
+        pytest.skip(kernel)
     w = inp["workload"]
     t = W.to_torch(inp)
     assert mla.wait_timeout_ns() == 2_000_000_000
@@ -230,7 +231,7 @@ def test_wait_timeout_expires_cleanly(mla, small_cases):
     try:
         assert mla.wait_timeout_ns() == 200
         out, lse = mla.decode(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], t["seq_lens"], w.scale,
-                              kernel="tcgen05")
+                              kernel=kernel)
         torch.cuda.synchronize()
     finally:
         mla.set_wait_timeout_ns(0)
@@ -245,7 +246,7 @@ def test_wait_timeout_expires_cleanly(mla, small_cases):
         for h in range(w.H):
             if np.isnan(l[b, 0, h]):
                 assert np.isnan(o[b, 0, h]).all()
-    o2, l2 = run_gpu(inp, "tcgen05", 0, tensors=t)
+    o2, l2 = run_gpu(inp, kernel, 0, tensors=t)
     compare(o2, l2, ref_o, ref_l, TOL[w.cache_dtype], "after the timeout")
 
 
