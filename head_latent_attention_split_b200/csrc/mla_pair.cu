@@ -58,7 +58,6 @@ constexpr uint32_t kPBytes = kRows * 128;              // P [128 rows][64 tokens
 constexpr uint32_t kMsgBytes = kPBytes + kRows * 8;    // + (rescale factor, 1 / row sum) per row
 constexpr int kStage = 4;                              // score CTA: outgoing message buffers
 constexpr int kRxBufs = 3;                             // output CTA: receive buffers
-constexpr int kPrefetchTiles = 6;                      // score CTA: L2 prefetch distance, in tiles
 
 constexpr uint32_t kOffRingS = 0;
 constexpr uint32_t kOffStage = kOffRingS + kSlotsS * kSlotBytesS;   // score CTA: outgoing messages
@@ -121,24 +120,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-
-// Walks the tiles of a worker's range in order (for the L2 prefetch that runs ahead of the loads).
-struct TileCursor {
-  SegmentIter it;
-  Segment sg;
-  int tile;
-  bool valid;
-  __device__ TileCursor(const SegmentIter& i) : it(i), tile(0), valid(false) {
-    valid = it.next(sg);
-    if (valid) tile = sg.tile_begin;
-  }
-  __device__ void advance() {
-    if (valid && ++tile >= sg.tile_end) {
-      valid = it.next(sg);
-      if (valid) tile = sg.tile_begin;
-    }
-  }
-};
 
 // Physical block of tile `tile` of sequence b; an id out of range sets the status word and
 // maps to the block just past the cache, which TMA reads as zeros.
@@ -232,27 +213,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (rank == 0 && warp == kProducerWarp) {
     // ------------------------------------------------------------------ score CTA: TMA producer
     if (lane == 0) {
+      // (An L2 prefetch of whole blocks a few tiles ahead of these loads measured slower on
+      // B200, the farther ahead the slower: the ring's own loads are the only reads.)
       SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
-      // Whole 72 KB blocks are prefetched into L2 kPrefetchTiles tiles ahead of the loads, so
-      // the ring's loads are L2 hits: the ring covers the L2 latency, not the HBM latency.
-      TileCursor pf(it);
-      const size_t block_bytes = (size_t)kBS * (kR + kDR) * 2;
-      auto prefetch_next = [&]() {
-        if (pf.valid) {
-          const int blk = __ldg(a.block_table + (size_t)pf.sg.b * a.max_blocks + pf.tile);
-          if (blk >= 0 && blk < a.num_blocks)
-            prefetch_l2((const uint8_t*)a.cache + (size_t)blk * block_bytes, (uint32_t)block_bytes);
-          pf.advance();
-        }
-      };
-      for (int i = 0; i < kPrefetchTiles; ++i) prefetch_next();
       Segment sg;
       uint32_t c = 0;   // slots issued
       bool ok = true;
       while (ok && it.next(sg)) {
         for (int tile = sg.tile_begin; ok && tile < sg.tile_end; tile += 2) {
           const int nt = min(2, sg.tile_end - tile);
-          for (int i = 0; i < nt; ++i) prefetch_next();
           const int blk0 = tile_block(a, sg.b, tile);
           const int blk1 = nt == 2 ? tile_block(a, sg.b, tile + 1) : 0;
 #pragma unroll 1   // rolled: see the score MMA loop

@@ -35,12 +35,3 @@ def compare(out, lse, ref_out, ref_lse, tol, what=""):
         lerr = np.abs(lse[~inf_ref] - ref_lse[~inf_ref]).max()
         assert lerr <= LSE_TOL, f"{what}: lse error {lerr:.3e}"
     return err
-
-
-def sample_rows(w, lens, n, seed):
-    """n (b, s, h) rows spread over the batch, including first/last sequence and head."""
-    rng = np.random.default_rng(seed)
-    rows = {(0, 0, 0), (w.B - 1, w.Sq - 1, w.H - 1)}
-    while len(rows) < n:
-        rows.add((int(rng.integers(w.B)), int(rng.integers(w.Sq)), int(rng.integers(w.H))))
-    return sorted(rows)
