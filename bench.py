@@ -74,13 +74,12 @@ def load_peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture of the tcgen05
-# decode kernel on a smaller batch of the same workload; profiles/) per cached token. A figure
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture of the decode
+# kernel the workload runs on a smaller batch of the same workload; profiles/) per cached token. A figure
 # only holds for the kernel sources it was taken on, keyed here by their SHA-256 prefix; for
 # any other source the bench reports traffic as null.
 MEASURED_TRAFFIC = {
-    "524335d759a92050": {"deepseek_v3": (304.125184e6 + 4.850944e6) / 262144,
-                         "fp8_cache": (169.770496e6 + 5.082368e6) / 262144},
+    "98163d24d61b8574": {"deepseek_v3": (304.293376e6 + 5.356800e6) / 262144},
 }
 KERNEL_SOURCES = ("mla_pair.cu", "mla_tc.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.h", "mla_tc.h")
 # The same for the sparse step's indexer (dram bytes per context token, batch 8 of the
@@ -101,7 +100,7 @@ def kernel_source_hash(files=KERNEL_SOURCES):
 
 def measured_traffic(wl, model, kernel):
     """Per-launch DRAM bytes of the decode kernel scaled from the ncu capture, or None."""
-    if kernel != "tcgen05":
+    if kernel not in ("tcgen05", "tc_pair"):
         return None
     per_tok = MEASURED_TRAFFIC.get(kernel_source_hash(), {}).get(wl.name)
     return None if per_tok is None else per_tok * model["tokens"]
