@@ -163,11 +163,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-// e4m3 pair (low byte = first code) -> two fp32, exact (hardware cvt to f16x2 first)
-__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two_codes) {
+// e4m3 pair (low byte = first code) -> f16x2, exact (every e4m3 value is an f16 value)
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   uint32_t h2;
   asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(h2) : "r"(two_codes));
-  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
+  return h2;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 template <bool kFp8, bool kSparse>
@@ -353,8 +359,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      // FP8 cache: the latent score MMAs and the PV run on fp16 operands (codes and P in fp16),
+      // the RoPE MMAs stay bf16
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, true);
+      constexpr uint32_t idesc_qk_lat = kFp8 ? idesc_f16_f32(128, 64, false) : idesc_qk;
+      constexpr uint32_t idesc_pv = kFp8 ? idesc_f16_f32(128, 256, true) : idesc_bf16_f32(128, 256, true);
       SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
       Segment sg;
       uint32_t g = 0, seg = 0;
@@ -394,7 +403,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
           for (int kk = 0; kk < 16; ++kk) {
             // latent channels [16 kk, 16 kk + 16): A = Q from TMEM, B = the cache chunk
             const uint64_t bdesc = smem_desc(base + (kk >> 2) * kKvLatChunk + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-            mma_ts(d, tmem + kTmemQ + 8 * kk, bdesc, idesc_qk, kk ? 1u : 0u);
+            mma_ts(d, tmem + kTmemQ + 8 * kk, bdesc, idesc_qk_lat, kk ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < (kFp8 ? 4 : 2); ++kk) {
@@ -459,7 +468,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
               *reinterpret_cast<uint4*>(lo_row + phys) = make_uint4(l[0], l[1], l[2], l[3]);
             }
           }
-          // codes of this token: 16 pieces of 16 bytes (channels [16 p, 16 p + 16)). Piece
+          // codes of this token -> fp16 (the latent MMAs' B operand): 16 pieces of 16 bytes
+          // (channels [16 p, 16 p + 16)). Piece
           // order is XOR-staggered by the token so that a warp's loads hit distinct banks.
           const uint8_t* src = base + 2 * kKvLatChunk + tok * 256;
           auto convert_piece = [&](const uint4 v, const int p) {
@@ -469,10 +479,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
             uint32_t o[8];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const float2 lo = e4m3x2_to_float2(wv[j] & 0xFFFFu);
-              const float2 hi = e4m3x2_to_float2(wv[j] >> 16);
-              o[2 * j] = pack_bf16x2(lo.x, lo.y);            // exact: e4m3 values fit bf16
-              o[2 * j + 1] = pack_bf16x2(hi.x, hi.y);
+              o[2 * j] = e4m3x2_to_f16x2(wv[j] & 0xFFFFu);   // exact: e4m3 values are f16 values
+              o[2 * j + 1] = e4m3x2_to_f16x2(wv[j] >> 16);
             }
             uint8_t* row = base + (p >> 2) * kKvLatChunk + tok * 128;
             const int p0 = 2 * (p & 3);
@@ -598,6 +606,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
           qv[4 * i + 2] = v.z;
           qv[4 * i + 3] = v.w;
         }
+        if constexpr (kFp8) {
+          // the latent score MMAs take fp16 operands: the bf16 query words to fp16 (exact for
+          // |q| in [2^-14, 65504] with at most 8 significant bits; smaller values lose bits)
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            qv[i] = pack_f16x2(__uint_as_float(qv[i] << 16), __uint_as_float(qv[i] & 0xFFFF0000u));
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_st16x2<64>(tmem + lane_off + kTmemQ + 16 * c, qv + 16 * c);
         tmem_wait_st();
@@ -702,7 +717,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
             const float p1 = any ? ex2_approx(x[k + 1] - m_run) : 0.f;
             psum += p0 + p1;
             if constexpr (kFp8)
-              pk[k >> 1] = pack_bf16x2(p0 * pcs[k], p1 * pcs[k + 1]);
+              pk[k >> 1] = pack_f16x2(p0 * pcs[k], p1 * pcs[k + 1]);   // the PV's fp16 A operand
             else
               pk[k >> 1] = pack_bf16x2(p0, p1);
           }

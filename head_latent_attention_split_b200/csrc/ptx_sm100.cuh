@@ -501,6 +501,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, bo
          | ((M >> 4) << 24);
 }
 
+// Instruction descriptor for kind::f16 with fp16 A/B and fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(uint32_t M, uint32_t N, bool b_mn_major) {
+  return (1u << 4)                   // D format: f32
+         | (0u << 7)                 // A format: f16
+         | (0u << 10)                // B format: f16
+         | ((b_mn_major ? 1u : 0u) << 16)
+         | ((N >> 3) << 17)
+         | ((M >> 4) << 24);
+}
+
 // Instruction descriptor for kind::f8f6f4 with e4m3 A/B (format code 0), both K-major,
 // fp32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N) {
