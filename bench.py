@@ -412,7 +412,7 @@ def dsa_arm(args, rank, local):
     idx = torch.empty((w.B, 1, k), dtype=torch.int32, device=dev)
     cnt = torch.empty((w.B, 1), dtype=torch.int32, device=dev)
     dp = mla.dsa_params_for(g["iq_codes"], g["ik_codes"], t["block_table"], L, k)
-    p = mla.params_for(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], w.scale, False, kernel="tcgen05")
+    p = mla.params_for(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], w.scale, False, kernel="auto")
     ws = torch.empty(max(1, mla.workspace_size(p)), dtype=torch.uint8, device=dev)
     out = torch.empty(t["q_lat"].shape, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(t["q_lat"].shape[:3], dtype=torch.float32, device=dev)

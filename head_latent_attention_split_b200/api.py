@@ -144,11 +144,11 @@ def dsa_topk(scores, seq_lens, top_k, causal=False, indices=None, counts=None, s
 
 
 def sparse_decode(q_lat, q_rope, kv_cache, block_table, indices, counts, softmax_scale, out=None, lse=None,
-                  workspace=None, num_workers=0, stream=None):
+                  workspace=None, num_workers=0, stream=None, kernel="auto"):
     """MLA decode over selected positions (q_len 1, bf16 cache): indices [B, top_k] (or
     [B, 1, top_k]) int32, counts [B] (or [B, 1]) int32. Returns (out, lse)."""
     import torch
-    p = params_for(q_lat, q_rope, kv_cache, block_table, softmax_scale, False, None, num_workers, "tcgen05")
+    p = params_for(q_lat, q_rope, kv_cache, block_table, softmax_scale, False, None, num_workers, kernel)
     top_k = indices.shape[-1]
     dev = q_lat.device
     if out is None:

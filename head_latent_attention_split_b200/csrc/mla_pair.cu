@@ -132,6 +132,25 @@ __device__ __forceinline__ int tile_block(const DecodeArgs& a, int b, int tile) 
   return blk;
 }
 
+// Physical cache row of entry j of sequence b's selected-token list (sparse decode). Entries
+// past the count, and entries whose position or block id is out of range (which also sets the
+// status word), map to the row just past the cache, which the row gathers read as zeros.
+__device__ __forceinline__ int sparse_row(const DecodeArgs& a, int b, int j, int count) {
+  const int oob = a.num_blocks * kBS;
+  if (j >= count) return oob;
+  const int t = __ldg(a.sel_idx + (size_t)b * a.top_k + j);
+  const int blk = (t >= 0 && t < a.max_blocks * kBS) ? __ldg(a.block_table + (size_t)b * a.max_blocks + t / kBS) : -1;
+  if (blk < 0 || blk >= a.num_blocks) {
+    set_status(a.status, MLA_ERR_BAD_BLOCK_ID);
+    return oob;
+  }
+  return blk * kBS + t % kBS;
+}
+
+// kSparse: tile t of a sequence is entries [64 t, 64 t + 64) of its selected-token list (the
+// sparse decode); tm_kv is then the cache as rows [num_blocks * 64][576] (one-row boxes of 64
+// channels, 128-byte swizzle) and the producers fetch each tile's rows with 4-row gathers.
+template <bool kSparse>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     pair_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_kv4,
                        const DecodeArgs a, const int n_rg,
@@ -210,7 +229,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const bool valid_row = grow < a.rows;
   const int s_idx = valid_row ? grow / a.H : 0;
 
-  if (rank == 0 && warp == kProducerWarp) {
+  if (kSparse && rank == 0 && warp == kProducerWarp) {
+    // ------------------------------------------------------------------ score CTA: row gathers
+    // lane L fetches rows 4L .. 4L + 3 of the tile pair (entries 64 tile + 4L + m), each of the
+    // slot's three 64-channel chunks with one 4-row gather: the same slot layout as the tiled
+    // loads (second tile's rows right after the first's).
+    SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
+    Segment sg;
+    uint32_t c = 0;   // slots issued
+    bool ok = true;
+    while (ok && it.next(sg)) {
+      for (int tile = sg.tile_begin; ok && tile < sg.tile_end; tile += 2) {
+        const int nt = min(2, sg.tile_end - tile);
+        const bool act = lane < 16 * nt;
+        int r4[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) r4[m] = act ? sparse_row(a, sg.b, tile * kBS + 4 * lane + m, sg.Lc) : 0;
+#pragma unroll 1   // rolled: see the score MMA loop
+        for (int g = 0; g < kChunksS / kGroupS; ++g, ++c) {
+          const uint32_t slot = c % kSlotsS;
+          bool free_slot = true;
+          if (lane == 0 && c >= (uint32_t)kSlotsS)
+            free_slot = mbar_wait<false>(smem_u32(&ctl.empty[slot]), ((c / kSlotsS) & 1) ^ 1, abort, timeout_ns);
+          ok = __shfl_sync(0xffffffffu, free_slot, 0);
+          if (!ok) break;
+          const uint32_t bar = smem_u32(&ctl.full[slot]);
+          const uint32_t dst = smem_u32(smem + kOffRingS + slot * kSlotBytesS);
+          if (lane == 0) mbar_arrive_expect_tx(bar, nt * kGroupS * kChunk);
+          __syncwarp();
+          if (act) {
+#pragma unroll
+            for (int jj = 0; jj < kGroupS; ++jj)
+              tma_gather4(dst + jj * kDChunk + lane * 512, &tm_kv, bar, 64 * (kGroupS * g + jj), r4);
+          }
+        }
+      }
+    }
+    if (lane == 0) {
+      int dummy = 0;
+      for (uint32_t i = 0; i < kSlotsS && i < c; ++i) {
+        const uint32_t cl = c - 1 - i;
+        mbar_wait<false>(smem_u32(&ctl.full[cl % kSlotsS]), (cl / kSlotsS) & 1, &dummy, drain_ns);
+      }
+      if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
+    }
+  } else if (rank == 0 && warp == kProducerWarp) {
     // ------------------------------------------------------------------ score CTA: TMA producer
     if (lane == 0) {
       // (An L2 prefetch of whole blocks a few tiles ahead of these loads measured slower on
@@ -512,6 +575,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
     }
+  } else if (kSparse && warp == kProducerWarp) {
+    // ------------------------------------------------------------------ output CTA: row gathers
+    // lanes 0-15 fetch the tile's rows 4L .. 4L + 3, each half stage's four 64-channel chunks
+    // with one 4-row gather each (the layout of the tiled 4-D box)
+    SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
+    Segment sg;
+    uint32_t h = 0;
+    bool ok = true;
+    while (ok && it.next(sg)) {
+      for (int tile = sg.tile_begin; ok && tile < sg.tile_end; ++tile) {
+        const bool act = lane < 16;
+        int r4[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) r4[m] = act ? sparse_row(a, sg.b, tile * kBS + 4 * lane + m, sg.Lc) : 0;
+#pragma unroll 1   // rolled: see the score MMA loop
+        for (int hc = 0; hc < 2; ++hc, ++h) {
+          const uint32_t hs = h % kHalvesO;
+          bool free_half = true;
+          if (lane == 0 && h >= (uint32_t)kHalvesO)
+            free_half = mbar_wait<false>(smem_u32(&ctl.oempty[hs]), ((h / kHalvesO) & 1) ^ 1, abort, timeout_ns);
+          ok = __shfl_sync(0xffffffffu, free_half, 0);
+          if (!ok) break;
+          const uint32_t bar = smem_u32(&ctl.ofull[hs]);
+          const uint32_t base = smem_u32(smem + kOffRingO + hs * kHalf);
+          if (lane == 0) mbar_arrive_expect_tx(bar, kHalf);
+          __syncwarp();
+          if (act) {
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+              tma_gather4(base + cc * kChunk + lane * 512, &tm_kv, bar, 256 * hc + 64 * cc, r4);
+          }
+        }
+      }
+    }
+    if (lane == 0) {
+      int dummy = 0;
+      for (uint32_t i = 0; i < kHalvesO && i < h; ++i) {
+        const uint32_t hl = h - 1 - i;
+        mbar_wait<false>(smem_u32(&ctl.ofull[hl % kHalvesO]), (hl / kHalvesO) & 1, &dummy, drain_ns);
+      }
+      if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
+    }
   } else if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ output CTA: TMA producer
     if (lane == 0) {
@@ -729,38 +834,60 @@ EncodeTiledFn encode_fn() {
 cudaError_t launch_pair_decode(const DecodeArgs& a, cudaStream_t s) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorInvalidValue;
-  // the cache [num_blocks][64][576] bf16, boxes of 64 channels x 64 tokens, 128-byte swizzle
-  CUtensorMap tm;
-  const cuuint64_t dims[3] = {(cuuint64_t)(kR + kDR), (cuuint64_t)kBS, (cuuint64_t)a.num_blocks};
-  const cuuint64_t strides[2] = {(cuuint64_t)(kR + kDR) * 2, (cuuint64_t)kBS * (kR + kDR) * 2};
-  const cuuint32_t box[3] = {64, (cuuint32_t)kBS, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.cache), dims, strides, box, estr,
-         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  // the same cache as (64 channels, 64 tokens, 9 channel chunks, blocks): one box = 4 chunks of a
-  // block, written as [chunk][token][128 bytes], the layout of four 3-D boxes side by side
-  CUtensorMap tm4;
-  const cuuint64_t dims4[4] = {64, (cuuint64_t)kBS, (cuuint64_t)(kR + kDR) / 64, (cuuint64_t)a.num_blocks};
-  const cuuint64_t strides4[3] = {(cuuint64_t)(kR + kDR) * 2, 128, (cuuint64_t)kBS * (kR + kDR) * 2};
-  const cuuint32_t box4[4] = {64, (cuuint32_t)kBS, 4, 1};
-  const cuuint32_t estr4[4] = {1, 1, 1, 1};
-  if (fn(&tm4, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(a.cache), dims4, strides4, box4, estr4,
-         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  static std::once_flag attr_once[64];
+  const bool sparse = a.sel_idx != nullptr;
+  if (sparse && (a.Sq != 1 || a.causal)) return cudaErrorInvalidValue;
+  CUtensorMap tm, tm4;
+  if (sparse) {
+    // the cache as rows [num_blocks * 64][576] bf16: one-row boxes of 64 channels (128 bytes,
+    // 128-byte swizzle) for 4-row gathers; rows past the cache read as zeros
+    const cuuint64_t dims[2] = {(cuuint64_t)(kR + kDR), (cuuint64_t)a.num_blocks * kBS};
+    const cuuint64_t strides[1] = {(cuuint64_t)(kR + kDR) * 2};
+    const cuuint32_t box[2] = {64, 1};
+    const cuuint32_t estr[2] = {1, 1};
+    if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.cache), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    tm4 = tm;   // unused by the gathering producers
+  } else {
+    // the cache [num_blocks][64][576] bf16, boxes of 64 channels x 64 tokens, 128-byte swizzle
+    const cuuint64_t dims[3] = {(cuuint64_t)(kR + kDR), (cuuint64_t)kBS, (cuuint64_t)a.num_blocks};
+    const cuuint64_t strides[2] = {(cuuint64_t)(kR + kDR) * 2, (cuuint64_t)kBS * (kR + kDR) * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kBS, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.cache), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    // the same cache as (64 channels, 64 tokens, 9 channel chunks, blocks): one box = 4 chunks of
+    // a block, written as [chunk][token][128 bytes], the layout of four 3-D boxes side by side
+    const cuuint64_t dims4[4] = {64, (cuuint64_t)kBS, (cuuint64_t)(kR + kDR) / 64, (cuuint64_t)a.num_blocks};
+    const cuuint64_t strides4[3] = {(cuuint64_t)(kR + kDR) * 2, 128, (cuuint64_t)kBS * (kR + kDR) * 2};
+    const cuuint32_t box4[4] = {64, (cuuint32_t)kBS, 4, 1};
+    const cuuint32_t estr4[4] = {1, 1, 1, 1};
+    if (fn(&tm4, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(a.cache), dims4, strides4, box4, estr4,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  static std::once_flag attr_once[2][64];
   int dev = 0;
   cudaGetDevice(&dev);
   cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once[dev & 63], [&] {
-    attr_err = cudaFuncSetAttribute(pair_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  std::call_once(attr_once[sparse ? 1 : 0][dev & 63], [&] {
+    attr_err = sparse ? cudaFuncSetAttribute(pair_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSmemBytes)
+                      : cudaFuncSetAttribute(pair_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSmemBytes);
   });
   if (attr_err != cudaSuccess) return attr_err;
   const int n_rg = (a.rows + kRows - 1) / kRows;
-  pair_decode_kernel<<<dim3(2 * a.W * n_rg), kThreads, kSmemBytes, s>>>(tm, tm4, a, n_rg, wait_timeout_ns(),
-                                                                        drain_timeout_ns());
+  const dim3 grid(2 * a.W * n_rg);
+  if (sparse)
+    pair_decode_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(tm, tm4, a, n_rg, wait_timeout_ns(), drain_timeout_ns());
+  else
+    pair_decode_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(tm, tm4, a, n_rg, wait_timeout_ns(),
+                                                                 drain_timeout_ns());
   return cudaGetLastError();
 }
 

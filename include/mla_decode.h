@@ -94,7 +94,7 @@ typedef enum {
   MLA_KERNEL_SIMT = 1,     /* fp32 CUDA-core kernel: any r <= 1024, r + d_r <= 1280 */
   MLA_KERNEL_TCGEN05 = 2,  /* tcgen05/TMA kernel: r = 512, d_r = 64, block_size = 64 */
   MLA_KERNEL_TC_PAIR = 3   /* split-role tcgen05/TMA kernel on CTA pairs (scores on one CTA, P.V on its
-                              peer): the shapes of MLA_KERNEL_TCGEN05 with a bf16 cache; dense decode only */
+                              peer): the shapes of MLA_KERNEL_TCGEN05 with a bf16 cache */
 } mla_kernel_t;
 
 typedef struct {
@@ -346,11 +346,12 @@ mla_status_t mla_dsa_index(const mla_dsa_params_t* params, const void* q_codes, 
 mla_status_t mla_dsa_topk(const mla_dsa_params_t* params, const float* scores, const int32_t* seq_lens,
                           int32_t* indices, int32_t* counts, void* stream);
 
-/* The decode's params (q_len 1, causal 0, BF16 cache, kernel AUTO or TCGEN05) and
+/* The decode's params (q_len 1, causal 0, BF16 cache, kernel AUTO, TC_PAIR or TCGEN05) and
  * workspace (mla_decode_workspace_size of the same params). indices [B, top_k] int32,
- * counts [B] int32, device; 0 <= counts[b] <= top_k is the caller's to guarantee (the kernel
- * reads indices[b, 0 .. counts[b]) and checks each position against the block table, not the
- * count against top_k; mla_dsa_topk's outputs satisfy it). */
+ * counts [B] int32, device. The kernel reads indices[b, 0 .. counts[b]) and checks each
+ * position against the block table; a count outside [0, top_k] is clamped into it and, like
+ * a bad position, sets the sticky status (MLA_ERR_BAD_SEQ_LEN / MLA_ERR_BAD_BLOCK_ID) and makes
+ * that sequence's rows NaN (mla_dsa_topk's outputs always satisfy it). */
 mla_status_t mla_sparse_decode(const mla_decode_params_t* params, int32_t top_k, const void* q_lat,
                                const void* q_rope, const void* kv_cache, const int32_t* block_table,
                                const int32_t* indices, const int32_t* counts, void* out, float* lse,

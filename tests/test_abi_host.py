@@ -265,7 +265,7 @@ def _sparse(m, **kw):
 
 
 @pytest.mark.parametrize("bad,code", [(dict(Sq=2), 2), (dict(causal=True), 2), (dict(cache_dtype=2), 2),
-                                      (dict(kernel="simt"), 2), (dict(kernel="tc_pair"), 2), (dict(top_k=0), 1), (dict(indices=None), 1),
+                                      (dict(kernel="simt"), 2), (dict(top_k=0), 1), (dict(indices=None), 1),
                                       (dict(counts=None), 1), (dict(q_rope=None), 1), (dict(workspace_bytes=16), 4),
                                       (dict(q_lat=FAKE + 8), 3), (dict(indices=FAKE + 2), 3)])
 def test_sparse_decode_rejects_bad_arguments_on_host(m, bad, code):

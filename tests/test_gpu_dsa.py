@@ -202,12 +202,15 @@ def test_topk_causal_rows():
 
 
 # ----------------------------------------------------------------------------- sparse decode
-def gpu_sparse(inp, idx, cnt):
+SPARSE_KERNELS = ["tcgen05", "tc_pair"]
+
+
+def gpu_sparse(inp, idx, cnt, kernel="auto"):
     mla = _mla()
     w = inp["workload"]
     t = W.to_torch(inp)
     out, lse = mla.sparse_decode(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], _dev(idx), _dev(cnt),
-                                 w.scale)
+                                 w.scale, kernel=kernel)
     _status_ok()
     return out.double().cpu().numpy(), lse.double().cpu().numpy()
 
@@ -218,19 +221,21 @@ def oracle_sparse(inp, idx, cnt):
                                 w.scale, idx.reshape(w.B, 1, -1), cnt.reshape(w.B, 1))
 
 
-def test_sparse_decode_on_the_oracle_selection(small):
+@pytest.mark.parametrize("kernel", SPARSE_KERNELS)
+def test_sparse_decode_on_the_oracle_selection(small, kernel):
     inp = small
     k = inp["top_k"]
     ref_scores = oracle_index(inp)
     n = oracle.attended_counts(inp["seq_lens"], 1, False)
     idx, cnt = oracle.dsa_topk(np.nan_to_num(ref_scores, nan=-np.inf), n, k)
     assert cnt.ravel().tolist() == [300, 512, 512]    # one row keeps all of its tokens
-    out, lse = gpu_sparse(inp, idx[:, 0], cnt[:, 0])
+    out, lse = gpu_sparse(inp, idx[:, 0], cnt[:, 0], kernel)
     ro, rl = oracle_sparse(inp, idx[:, 0], cnt[:, 0])
     compare(out, lse, ro, rl, TOL[W.BF16], "sparse decode")
 
 
-def test_sparse_decode_random_lists_and_edges(small):
+@pytest.mark.parametrize("kernel", SPARSE_KERNELS)
+def test_sparse_decode_random_lists_and_edges(small, kernel):
     inp = small
     rng = np.random.default_rng(11)
     k = 200
@@ -240,13 +245,14 @@ def test_sparse_decode_random_lists_and_edges(small):
     for b in range(3):
         if cnt[b]:
             idx[b, :cnt[b]] = rng.choice(int(lens[b]), size=int(cnt[b]), replace=False)   # any order
-    out, lse = gpu_sparse(inp, idx, cnt)
+    out, lse = gpu_sparse(inp, idx, cnt, kernel)
     ro, rl = oracle_sparse(inp, idx, cnt)
     assert np.all(out[0] == 0) and np.all(np.isneginf(lse[0]))
     compare(out, lse, ro, rl, TOL[W.BF16], "sparse decode, random lists")
 
 
-def test_sparse_decode_every_token_is_dense(small):
+@pytest.mark.parametrize("kernel", SPARSE_KERNELS)
+def test_sparse_decode_every_token_is_dense(small, kernel):
     # a list holding every position equals the dense decode (the oracle's dense decode)
     inp = small
     lens = inp["seq_lens"]
@@ -254,7 +260,7 @@ def test_sparse_decode_every_token_is_dense(small):
     idx = np.full((3, k), -1, np.int32)
     for b in range(3):
         idx[b, :lens[b]] = np.arange(lens[b])
-    out, lse = gpu_sparse(inp, idx, lens.astype(np.int32))
+    out, lse = gpu_sparse(inp, idx, lens.astype(np.int32), kernel)
     ro, rl = oracle.decode_inputs(inp)
     compare(out, lse, ro, rl, TOL[W.BF16], "sparse == dense")
 
