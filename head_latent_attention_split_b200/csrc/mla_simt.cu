@@ -236,22 +236,60 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const DecodeArgs a) {
   for (int i = lane; i < splits; i += 32) Z += expf(a.lse_part[(slot0 + i) * a.rows + row] - M);
   Z = warp_sum(Z);
   const float lse_v = M + logf(Z);
-  for (int k0 = 0; k0 < a.r; k0 += 32 * 4) {
-    float o[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int i = 0; i < splits; ++i) {
-      const size_t prow = (slot0 + i) * a.rows + row;
-      const float wgt = expf(a.lse_part[prow] - lse_v);
-      if (wgt == 0.f) continue;
+  if (a.r % 4 == 0) {
+    // 512 channels per pass, 16 per lane as four float4 pieces; each split's pieces are
+    // independent loads, so a split costs one memory latency, not one per piece
+    for (int k0 = 0; k0 < a.r; k0 += 512) {
+      float4 o[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) o[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+      for (int i = 0; i < splits; ++i) {
+        const size_t prow = (slot0 + i) * a.rows + row;
+        const float wgt = expf(a.lse_part[prow] - lse_v);
+        if (wgt == 0.f) continue;
+        const float* src = a.o_part + prow * a.r;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int k = k0 + 4 * lane + 128 * u;
+          if (k < a.r) {
+            const float4 v = *reinterpret_cast<const float4*>(src + k);
+            o[u].x = fmaf(wgt, v.x, o[u].x);
+            o[u].y = fmaf(wgt, v.y, o[u].y);
+            o[u].z = fmaf(wgt, v.z, o[u].z);
+            o[u].w = fmaf(wgt, v.w, o[u].w);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int k = k0 + 4 * lane + 128 * u;
+        if (k < a.r) {
+          store_out(a.out, a.out_dtype, orow * a.r + k, o[u].x);
+          store_out(a.out, a.out_dtype, orow * a.r + k + 1, o[u].y);
+          store_out(a.out, a.out_dtype, orow * a.r + k + 2, o[u].z);
+          store_out(a.out, a.out_dtype, orow * a.r + k + 3, o[u].w);
+        }
+      }
+    }
+  } else {
+    for (int k0 = 0; k0 < a.r; k0 += 32 * 4) {
+      float o[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int i = 0; i < splits; ++i) {
+        const size_t prow = (slot0 + i) * a.rows + row;
+        const float wgt = expf(a.lse_part[prow] - lse_v);
+        if (wgt == 0.f) continue;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int k = k0 + lane + 32 * u;
+          if (k < a.r) o[u] = fmaf(wgt, a.o_part[prow * a.r + k], o[u]);
+        }
+      }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int k = k0 + lane + 32 * u;
-        if (k < a.r) o[u] = fmaf(wgt, a.o_part[prow * a.r + k], o[u]);
+        if (k < a.r) store_out(a.out, a.out_dtype, orow * a.r + k, o[u]);
       }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int k = k0 + lane + 32 * u;
-      if (k < a.r) store_out(a.out, a.out_dtype, orow * a.r + k, o[u]);
     }
   }
   if (lane == 0) a.lse[orow] = lse_v;
