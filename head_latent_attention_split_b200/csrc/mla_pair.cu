@@ -1,5 +1,6 @@
 // Split-role tensor-core (tcgen05 + TMA) absorbed-MLA decode for r = 512, d_r = 64, 64-token
-// cache blocks, bf16 queries and a bf16 cache.
+// cache blocks, bf16 queries and a bf16 cache; dense token ranges, or (kSparse) each sequence's
+// list of selected positions.
 //
 // The fp32 output of 128 query rows over all 512 latent channels, O[128 x 512], fills the 512
 // TMEM columns of one SM, so a decode worker is a cluster of two CTAs. The roles differ:
@@ -7,23 +8,25 @@
 //   score CTA (cluster rank 0): streams every tile of the worker's range whole (512 latent +
 //     64 RoPE channels) and computes full scores S = Q . C^T with tcgen05: A = the absorbed
 //     query held in TMEM, B = the cache rows in shared memory. Tiles are scored two at a time
-//     (N = 128 tokens per MMA): a tcgen05 MMA costs about the same ~60-70 cycles for N = 64
-//     and N = 128 on B200, so pairs of tiles double the score rate. Eight softmax warps (two
-//     per SM sub-partition: warp q takes the first tile's 64 columns of rows [32q, 32q + 32),
-//     warp q + 4 the second tile's) run the online softmax in registers, thread = query row,
-//     share the row maximum through shared memory, and send each tile's bf16 probabilities
-//     P[128 x 64] plus one rescale factor per row to the output CTA with bulk copies over
-//     distributed shared memory.
-//   output CTA (cluster rank 1): streams the same tiles' 512 latent channels (the second read of
-//     each tile is served by L2), rescales O rows whose running maximum moved, and accumulates
-//     O[128 x 512] += P . C with tcgen05 (A = P in shared memory, B = the tile read N-major,
-//     N = 256), then normalises O into the output (or the split partial).
+//     (N = 128 tokens per MMA): on B200 a tcgen05 MMA costs ~60 cycles up to N = 64 and ~70 at
+//     N = 128, so pairs of tiles nearly double the score rate. The cache ring is 3 slots of
+//     48 KB, each three 64-channel chunks of both tiles of a pair (6 TMA boxes per barrier).
+//     Eight softmax warps (two per SM sub-partition: warp q takes the first tile's 64 columns
+//     of rows [32q, 32q + 32), warp q + 4 the second tile's) run the online softmax in
+//     registers, thread = query row, share the row maximum through shared memory, and write
+//     each tile's message (bf16 P[128 x 64] as K-major core matrices plus one rescale factor
+//     and 1/row-sum per row, 17 KB) into one of four staging buffers; a post warp sends each
+//     message with one bulk copy into the output CTA's shared memory.
+//   output CTA (cluster rank 1): streams the same tiles' 512 latent channels (one 4-D TMA box per
+//     256 channels; the second read of each tile is served by L2), rescales O rows whose
+//     running maximum moved, and accumulates O[128 x 512] += P . C with tcgen05 (A = P in
+//     shared memory, B = the tile read N-major, N = 256), then normalises O into the output
+//     (or the split partial).
 //
-// Only P crosses between the SMs, in one direction (17 KB per tile, three receive buffers); the
-// completion of the PV that read a receive buffer is signalled straight to the score CTA by the
-// tensor core (a commit arriving on the score CTA's barrier), so there is no round trip on the
-// per-tile path. The score CTA's cache ring is 11 slots of 16 KB, each the same 64-channel chunk
-// of the two tiles of a pair, released chunk by chunk as the score MMAs finish reading it.
+// Only P crosses between the SMs, in one direction. The completion of the PV that read a
+// receive buffer is signalled straight to the score CTA by the tensor core (a commit arriving on
+// the score CTA's barrier), and the output CTA hands a staging buffer back with one remote
+// arrive once its message has landed, so no thread waits on a round trip per tile.
 //
 // The running maximum of a row only moves when a tile pair raises it by more than 2^8 (log2
 // units), so O is rescaled rarely; the softmax uses base-2 exponentials of scale * log2(e) *
@@ -130,6 +133,16 @@ __device__ __forceinline__ int tile_block(const DecodeArgs& a, int b, int tile) 
     return a.num_blocks;
   }
   return blk;
+}
+
+// Prefetch into L2 the query rows of row group rg of sequence b (latent and RoPE parts), so the
+// softmax warps' loads of a new segment's query hit L2: the score MMAs wait for them.
+__device__ __forceinline__ void prefetch_query(const DecodeArgs& a, int b, int rg) {
+  const int r0 = rg * kRows, nr = min(kRows, a.rows - r0);
+  if (nr <= 0) return;
+  const size_t row = (size_t)b * a.rows + r0;
+  prefetch_l2((const uint16_t*)a.q_lat + row * kR, (uint32_t)nr * kR * 2);
+  prefetch_l2((const uint16_t*)a.q_rope + row * kDR, (uint32_t)nr * kDR * 2);
 }
 
 // Physical cache row of entry j of sequence b's selected-token list (sparse decode). Entries
@@ -239,6 +252,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t c = 0;   // slots issued
     bool ok = true;
     while (ok && it.next(sg)) {
+      if (lane == 0) prefetch_query(a, sg.b, rg);
       for (int tile = sg.tile_begin; ok && tile < sg.tile_end; tile += 2) {
         const int nt = min(2, sg.tile_end - tile);
         const bool act = lane < 16 * nt;
@@ -283,6 +297,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t c = 0;   // slots issued
       bool ok = true;
       while (ok && it.next(sg)) {
+        prefetch_query(a, sg.b, rg);
         for (int tile = sg.tile_begin; ok && tile < sg.tile_end; tile += 2) {
           const int nt = min(2, sg.tile_end - tile);
           const int blk0 = tile_block(a, sg.b, tile);

@@ -56,35 +56,10 @@ __device__ __forceinline__ void mbar_arrive_remote_cta(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
-// Arrive on an mbarrier of another CTA of the cluster with release at cluster scope: the
-// writes that happen before this arrival (this thread's, and those it acquired) are visible to
-// a thread that completes a wait on that barrier with acquire at cluster scope.
-__device__ __forceinline__ void mbar_arrive_remote_cluster(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
-}
-
 // Arrive on an mbarrier of another CTA of the cluster, relaxed (no ordering of earlier memory
 // operations): a signal whose only payload is the arrival itself, or one that follows a fence.
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
-}
-
-__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
-
-// Global loads cached in L2 only (the line may have been rewritten by another SM since this
-// SM last read it).
-__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p)
-               : "memory");
-  return v;
-}
-__device__ __forceinline__ float2 ld_cg_v2f(const void* p) {
-  float2 v;
-  asm volatile("ld.global.cg.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p) : "memory");
-  return v;
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
@@ -163,26 +138,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// Bounded wait that polls without suspending (for short waits on the critical path, where a
-// suspended thread may resume later than the phase completes). Same contract as mbar_wait.
-template <bool kCluster>
-__device__ __forceinline__ bool mbar_spin(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t timeout_ns) {
-  uint64_t t0 = 0;
-  for (uint32_t it = 0;; ++it) {
-    if (kCluster ? mbar_test_wait_cluster(bar, parity) : mbar_test_wait(bar, parity)) return true;
-    if ((it & 255u) == 255u) {
-      if (*abort) return false;
-      const uint64_t now = globaltimer();
-      if (t0 == 0) {
-        t0 = now;
-      } else if (now - t0 > timeout_ns) {
-        *abort = 1;
-        return false;
-      }
-    }
-  }
-}
-
 // ------------------------------------------------------------------------ cluster / DSMEM
 __device__ __forceinline__ uint32_t mapa(uint32_t smem_addr, uint32_t rank) {
   uint32_t r;
@@ -201,16 +156,6 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
       : "memory");
 }
 
-// Bulk copy global -> this CTA's shared memory, completing on a local mbarrier (tx bytes).
-// Addresses 16-byte aligned, size a multiple of 16.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
-
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Wait until at most N committed bulk groups of this thread still read their source.
@@ -222,21 +167,6 @@ __device__ __forceinline__ void bulk_wait_group_read() {
 __device__ __forceinline__ void st_async_b32(uint32_t cluster_addr, uint32_t v, uint32_t cluster_bar) {
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(cluster_addr),
                "r"(v), "r"(cluster_bar)
-               : "memory");
-}
-
-// 16 and 8 bytes into another CTA's shared memory, completing that many bytes on its mbarrier.
-__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                                            uint32_t cluster_bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                   cluster_addr),
-               "r"(a), "r"(b), "r"(c), "r"(d), "r"(cluster_bar)
-               : "memory");
-}
-
-__device__ __forceinline__ void st_async_v2f(uint32_t cluster_addr, float a, float b, uint32_t cluster_bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(cluster_addr),
-               "f"(a), "f"(b), "r"(cluster_bar)
                : "memory");
 }
 
@@ -446,9 +376,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
       "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
-
-// Every bulk copy this thread committed has completed (destination writes included).
-__device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ------------------------------------------------------------------------ descriptors
 // Shared-memory matrix descriptor (sm_100 format): start address, leading and stride
