@@ -238,7 +238,12 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const DecodeArgs a) {
   const float lse_v = M + logf(Z);
   if (a.r % 4 == 0) {
     // 512 channels per pass, 16 per lane as four float4 pieces; each split's pieces are
-    // independent loads, so a split costs one memory latency, not one per piece
+    // independent loads, so a split costs one memory latency, not one per piece. The split
+    // weights come from lane i (splits <= 32) by shuffle; the output goes out 4 channels per store.
+    const float wl = lane < splits ? expf(a.lse_part[(slot0 + lane) * a.rows + row] - lse_v) : 0.f;
+    // 4 output channels per store when the output allows it (the SIMT path takes 4-byte
+    // aligned outputs)
+    const bool vec_out = ((uintptr_t)a.out % (a.out_dtype == kF32 ? 16u : 8u)) == 0;
     for (int k0 = 0; k0 < a.r; k0 += 512) {
       float4 o[4];
 #pragma unroll
@@ -246,7 +251,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const DecodeArgs a) {
 #pragma unroll 2
       for (int i = 0; i < splits; ++i) {
         const size_t prow = (slot0 + i) * a.rows + row;
-        const float wgt = expf(a.lse_part[prow] - lse_v);
+        const float wgt = i < 32 ? __shfl_sync(0xffffffffu, wl, i) : expf(a.lse_part[prow] - lse_v);
         if (wgt == 0.f) continue;
         const float* src = a.o_part + prow * a.r;
 #pragma unroll
@@ -264,11 +269,22 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const DecodeArgs a) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int k = k0 + 4 * lane + 128 * u;
-        if (k < a.r) {
-          store_out(a.out, a.out_dtype, orow * a.r + k, o[u].x);
-          store_out(a.out, a.out_dtype, orow * a.r + k + 1, o[u].y);
-          store_out(a.out, a.out_dtype, orow * a.r + k + 2, o[u].z);
-          store_out(a.out, a.out_dtype, orow * a.r + k + 3, o[u].w);
+        if (k < a.r && !vec_out) {
+          const size_t e = orow * a.r + k;
+          store_out(a.out, a.out_dtype, e, o[u].x);
+          store_out(a.out, a.out_dtype, e + 1, o[u].y);
+          store_out(a.out, a.out_dtype, e + 2, o[u].z);
+          store_out(a.out, a.out_dtype, e + 3, o[u].w);
+        } else if (k < a.r) {
+          const size_t e = orow * a.r + k;
+          if (a.out_dtype == kF32) {
+            *reinterpret_cast<float4*>((float*)a.out + e) = o[u];
+          } else {
+            uint32_t lo, hi;   // round to nearest even; NaN stays NaN
+            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(o[u].y), "f"(o[u].x));
+            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(o[u].w), "f"(o[u].z));
+            *reinterpret_cast<uint2*>((uint16_t*)a.out + e) = make_uint2(lo, hi);
+          }
         }
       }
     }
