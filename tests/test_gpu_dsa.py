@@ -332,13 +332,14 @@ def test_full_size_sampled_rows(full):
     rng = np.random.default_rng(21)
     lst = np.stack([np.sort(rng.choice(int(L), size=k, replace=False)) for L in inp["seq_lens"]]).astype(np.int32)
     cnts = np.full(w.B, k, np.int32)
-    out, lse = gpu_sparse(inp, lst, cnts)
+    outs = {kern: gpu_sparse(inp, lst, cnts, kern) for kern in SPARSE_KERNELS}
     for b in rows:
         sub = {key: inp[key] for key in ("kv_cache", "k_rope_cache", "kv_scale")}
         ro, rl = oracle.decode_sparse(inp["q_lat"][b:b + 1], inp["q_rope"][b:b + 1], sub["kv_cache"],
                                       inp["block_table"][b:b + 1], inp["seq_lens"][b:b + 1], w.scale,
                                       lst[b:b + 1].reshape(1, 1, k), cnts[b:b + 1].reshape(1, 1))
-        compare(out[b:b + 1], lse[b:b + 1], ro, rl, TOL[W.BF16], f"full-size sparse decode b={b}")
+        for kern, (out, lse) in outs.items():
+            compare(out[b:b + 1], lse[b:b + 1], ro, rl, TOL[W.BF16], f"full-size sparse decode ({kern}) b={b}")
 
 
 # ----------------------------------------------------------------------------- error paths
@@ -376,7 +377,8 @@ def test_index_bad_block_id_and_seq_len_set_status(small):
     assert cnt.cpu().numpy()[2, 0] == 0 and (idx.cpu().numpy()[2] == -1).all()
 
 
-def test_sparse_decode_bad_position_sets_status(small):
+@pytest.mark.parametrize("kernel", SPARSE_KERNELS)
+def test_sparse_decode_bad_position_sets_status(small, kernel):
     """A listed position outside the block table's range sets MLA_ERR_BAD_BLOCK_ID and turns that
     sequence's rows NaN; the other sequences are unaffected."""
     torch = _torch()
@@ -391,7 +393,7 @@ def test_sparse_decode_bad_position_sets_status(small):
     w = inp["workload"]
     t = W.to_torch(inp)
     out, lse = mla.sparse_decode(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], _dev(bad), _dev(cnt),
-                                 w.scale)
+                                 w.scale, kernel=kernel)
     torch.cuda.synchronize()
     assert mla.device_status() == 6
     o, l = out.double().cpu().numpy(), lse.double().cpu().numpy()
@@ -401,7 +403,8 @@ def test_sparse_decode_bad_position_sets_status(small):
     compare(o[keep], l[keep], ro[keep], rl[keep], TOL[W.BF16], "sequences without the bad position")
 
 
-def test_sparse_decode_count_above_top_k_sets_status(small):
+@pytest.mark.parametrize("kernel", SPARSE_KERNELS)
+def test_sparse_decode_count_above_top_k_sets_status(small, kernel):
     """A count above top_k (the list's row stride) is an error: MLA_ERR_BAD_SEQ_LEN, that
     sequence's rows NaN, nothing read past its list; the other sequences are unaffected."""
     torch = _torch()
@@ -416,7 +419,7 @@ def test_sparse_decode_count_above_top_k_sets_status(small):
     w = inp["workload"]
     t = W.to_torch(inp)
     out, lse = mla.sparse_decode(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], _dev(idx), _dev(bad),
-                                 w.scale)
+                                 w.scale, kernel=kernel)
     torch.cuda.synchronize()
     assert mla.device_status() == 7
     o, l = out.double().cpu().numpy(), lse.double().cpu().numpy()
