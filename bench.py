@@ -76,12 +76,15 @@ def load_peaks():
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture of the decode
 # kernel the workload runs on a smaller batch of the same workload; profiles/) per cached token. A figure
-# only holds for the kernel sources it was taken on, keyed here by their SHA-256 prefix; for
-# any other source the bench reports traffic as null.
+# only holds for the sources the kernel was built from, keyed here by kernel and the SHA-256 prefix of
+# those files; for any other source the bench reports traffic as null.
 MEASURED_TRAFFIC = {
-    "df5d01e6da87d6d1": {"deepseek_v3": (304.350976e6 + 4.457728e6) / 262144},
+    ("tc_pair", "c34dd76ad94899ec"): {"deepseek_v3": (304.350976e6 + 4.457728e6) / 262144},
 }
-KERNEL_SOURCES = ("mla_pair.cu", "mla_tc.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.h", "mla_tc.h")
+KERNEL_SOURCES = {
+    "tc_pair": ("mla_pair.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.h", "mla_tc.h"),
+    "tcgen05": ("mla_tc.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.h", "mla_tc.h"),
+}
 # The same for the sparse step's indexer (dram bytes per context token, batch 8 of the
 # 128K workload), keyed by the sources of mla_dsa.cu and its headers.
 DSA_TRAFFIC = {
@@ -90,7 +93,7 @@ DSA_TRAFFIC = {
 DSA_SOURCES = ("mla_dsa.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.h")
 
 
-def kernel_source_hash(files=KERNEL_SOURCES):
+def kernel_source_hash(files):
     h = hashlib.sha256()
     for f in files:
         with open(os.path.join(ROOT, "head_latent_attention_split_b200", "csrc", f), "rb") as fh:
@@ -102,7 +105,7 @@ def measured_traffic(wl, model, kernel):
     """Per-launch DRAM bytes of the decode kernel scaled from the ncu capture, or None."""
     if kernel not in ("tcgen05", "tc_pair"):
         return None
-    per_tok = MEASURED_TRAFFIC.get(kernel_source_hash(), {}).get(wl.name)
+    per_tok = MEASURED_TRAFFIC.get((kernel, kernel_source_hash(KERNEL_SOURCES[kernel])), {}).get(wl.name)
     return None if per_tok is None else per_tok * model["tokens"]
 
 

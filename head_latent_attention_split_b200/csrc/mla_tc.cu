@@ -51,9 +51,10 @@
 //    lesson, Chapter 7 "DSA runs in MLA's MQA mode"): the same kernel over each
 //    sequence's list of selected positions instead of its whole length. The per-sequence
 //    length is the list's count, and tile t holds list entries [64 t, 64 t + 64); the
-//    producer warp maps them through the block table and fetches the 64 token rows of
-//    the CTA's channel slice with TMA row gathers (four rows per load), into the same
-//    swizzled stage layout. Entries past the count read as zeros.
+//    producer warp maps them through the block table and copies the 64 token rows of
+//    the CTA's channel slice with 16-byte cp.async copies (one 512-byte row slice per warp
+//    instruction) into the same swizzled stage layout; each lane's copies complete one
+//    arrival on the stage barrier. Entries past the count are zero-filled without a read.
 // The work split over workers (CTA pairs) is the flat block list plan of mla_device.cuh.
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -170,6 +171,18 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   return h2;
 }
 
+// 16-byte global -> shared copy that bypasses L1 (LDGSTS). src_bytes = 0 reads nothing and
+// writes 16 zero bytes.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// One arrival on the mbarrier once every cp.async this thread issued before has completed
+// (noinc: the arrival counts against the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -199,7 +212,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_u32(&ctl.kv_full[i]), 1);
+      mbar_init(smem_u32(&ctl.kv_full[i]), kSparse ? 32 : 1);   // sparse: one cp.async arrival per lane
       mbar_init(smem_u32(&ctl.kv_empty[i]), 1);
     }
     mbar_init(smem_u32(&ctl.q_full), 1 + kSoftmaxThreads);   // RoPE part by TMA + latent part into TMEM
@@ -247,14 +260,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
   const WorkerPlan plan = ctl.plan;
 
   if (kSparse && warp == kProducerWarp) {
-    // ------------------------------------------------------------------ gather producer (sparse)
-    // Lanes map the 64 listed positions of a tile to cache rows (two each); lane l < 16
-    // then loads rows 4 l .. 4 l + 3 of every channel chunk with one row gather each.
+    // ------------------------------------------------------------------ copy producer (sparse)
+    // Lanes map the 64 listed positions of a tile to cache rows (two each; -1 = no row). Each
+    // cache row is then copied by the whole warp with 16-byte cp.async copies into the same
+    // swizzled stage layout the TMA path writes: lane l takes unit l of the row's 512-byte
+    // latent slice (one row per warp instruction), and one 16-byte unit of eight rows' 64-byte
+    // RoPE slices. Every lane's copies of a tile complete one arrival on the stage barrier;
+    // rows that are not there are zero-filled without a read.
     SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
     Segment sg;
     uint32_t g = 0, seg = 0;
     bool ok = true;
-    const int oob_row = a.num_blocks * kBS;   // past the last row: the load fills zeros
+    const char* cache = static_cast<const char*>(a.cache);
+    constexpr uint32_t kRowBytes = (kR + kDR) * 2;
+    const uint32_t lat_src = 512 * rank + 16 * lane;                  // byte offset in a cache row
+    const uint32_t lat_dst = (lane >> 3) * kKvLatChunk;               // 64-channel chunk of the unit
+    const uint32_t rope_src = 2 * kR + 64 * rank + 16 * (lane & 3);
     while (ok && it.next(sg)) {
       if (lane == 0) {
         ok = mbar_wait<false>(smem_u32(&ctl.q_empty), (seg & 1) ^ 1, abort, timeout_ns);
@@ -271,7 +292,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int j = tile * kBS + 32 * hh + lane;   // list entry
-          int row = oob_row;
+          int row = -1;
           if (j < sg.Lc) {
             const int t = __ldg(a.sel_idx + (size_t)sg.b * a.top_k + j);
             const int blk = (t >= 0 && t < a.max_blocks * kBS) ? __ldg(a.block_table + (size_t)sg.b * a.max_blocks + t / kBS) : -1;
@@ -282,30 +303,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
           }
           rw[hh] = row;
         }
-        int r4[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int i = 4 * lane + m;   // token row of the tile (meaningful for lanes < 16)
-          const int v0 = __shfl_sync(0xffffffffu, rw[0], i & 31);
-          const int v1 = __shfl_sync(0xffffffffu, rw[1], i & 31);
-          r4[m] = i < 32 ? v0 : v1;
-        }
         const uint32_t st = g % kStages, ph = (g / kStages) & 1;
         if (lane == 0) ok = mbar_wait<false>(smem_u32(&ctl.kv_empty[st]), ph ^ 1, abort, timeout_ns);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        const uint32_t bar = smem_u32(&ctl.kv_full[st]);
         const uint32_t base = sKv + st * kStageBytes;
-        if (lane == 0) mbar_arrive_expect_tx(bar, kStageBytes);
-        __syncwarp();
-        if (lane < 16) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) tma_gather4(base + c * kKvLatChunk + lane * 512, &tm_kv, bar, 256 * rank + 64 * c, r4);
-          tma_gather4(base + 4 * kKvLatChunk + lane * 256, &tm_kr, bar, kR + 32 * rank, r4);
+        for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll 8
+          for (int ii = 0; ii < 32; ++ii) {
+            const int i = 32 * hh + ii;
+            const int row = __shfl_sync(0xffffffffu, rw[hh], ii);
+            const char* src = cache + (size_t)(row < 0 ? 0 : row) * kRowBytes + lat_src;
+            cp_async_16(base + lat_dst + i * 128 + (((lane & 7) ^ (i & 7)) << 4), src, row < 0 ? 0u : 16u);
+          }
         }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int i = 8 * k + (lane >> 2);                 // rows 8k .. 8k + 7, four lanes each
+          const int row = __shfl_sync(0xffffffffu, rw[k >> 2], i & 31);
+          const char* src = cache + (size_t)(row < 0 ? 0 : row) * kRowBytes + rope_src;
+          cp_async_16(base + 4 * kKvLatChunk + i * 64 + (((lane & 3) ^ ((i >> 1) & 3)) << 4), src, row < 0 ? 0u : 16u);
+        }
+        cp_async_arrive_noinc(smem_u32(&ctl.kv_full[st]));
       }
       ++seg;
     }
+    cp_async_wait_all();
     if (lane == 0) {
       int dummy = 0;
       for (uint32_t i = 0; i < kStages && i < g; ++i) {
@@ -397,6 +421,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
                mbar_wait<false>(smem_u32(&ctl.s_empty), (g & 1) ^ 1, abort, timeout_ns);
           if (!ok) break;
           tc_fence_after();
+          if constexpr (kSparse) fence_proxy_async_smem();   // the tile was written by cp.async
           const uint32_t base = sKv + st * kStageBytes;
           const uint32_t d = tmem + kTmemS;
 #pragma unroll
@@ -985,20 +1010,6 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D tensor map with a one-row box, for row gathers: dims (inner, rows), row stride s1.
-bool make_map_2d_rows(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t s1, uint32_t b0,
-                      CUtensorMapSwizzle sw) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {d0, d1};
-  const cuuint64_t strides[1] = {s1};
-  const cuuint32_t box[2] = {b0, 1};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int row_groups(int rows) { return (rows + kRows - 1) / kRows; }
 
 }  // namespace
@@ -1025,10 +1036,7 @@ cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
   if (sparse && (fp8 || a.Sq != 1 || a.causal)) return cudaErrorInvalidValue;
   bool ok = make_map_3d(&tqr, a.q_rope, kDR, rows, a.B, kDR * 2, rows * kDR * 2, 32, kRows, CU_TENSOR_MAP_SWIZZLE_64B);
   if (sparse) {
-    // the cache as rows [num_blocks * 64][576] bf16: 64-channel latent boxes, 32-channel RoPE boxes
-    const uint64_t nrows = (uint64_t)a.num_blocks * kBS;
-    ok = ok && make_map_2d_rows(&tkv, a.cache, kR + kDR, nrows, (kR + kDR) * 2, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_map_2d_rows(&tkr, a.cache, kR + kDR, nrows, (kR + kDR) * 2, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+    tkv = tkr = tqr;   // the sparse kernel copies cache rows with cp.async; no cache maps
   } else if (fp8) {
     // codes [num_blocks][64][512] e4m3 (256-byte boxes, no swizzle), RoPE keys [num_blocks][64][64] bf16
     ok = ok &&
