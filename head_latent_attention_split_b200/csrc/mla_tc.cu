@@ -122,10 +122,10 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kSoftmaxThreads = 256;  // warps 0-7
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kConvWarp0 = 10;        // FP8 cache only: warps 10-11 decode codes in place
+constexpr int kConvWarp0 = 10;        // FP8 cache: warps 10-11 decode codes in place; sparse: warp 10 copies
 constexpr int kConvThreads = 64;      // one thread per token row of a tile
-template <bool kFp8>
-constexpr int threads_for() { return kFp8 ? 384 : 320; }
+template <bool kFp8, bool kSparse>
+constexpr int threads_for() { return kFp8 ? 384 : kSparse ? 352 : 320; }
 constexpr uint32_t kFp8CodeBytes = kBS * 256;                    // this CTA's codes of one block
 constexpr uint32_t kFp8StageTx = kFp8CodeBytes + kKvRope + kBS * 4;   // codes, RoPE key, scales
 
@@ -190,7 +190,7 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 }
 
 template <bool kFp8, bool kSparse>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(), 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8, kSparse>(), 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_sc,
                      const DecodeArgs a, const int n_rg, const uint64_t timeout_ns, const uint64_t drain_ns) {
@@ -212,7 +212,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(smem_u32(&ctl.kv_full[i]), kSparse ? 32 : 1);   // sparse: one cp.async arrival per lane
+      mbar_init(smem_u32(&ctl.kv_full[i]), kSparse ? 64 : 1);   // sparse: one cp.async arrival per copy lane
       mbar_init(smem_u32(&ctl.kv_empty[i]), 1);
     }
     mbar_init(smem_u32(&ctl.q_full), 1 + kSoftmaxThreads);   // RoPE part by TMA + latent part into TMEM
@@ -259,14 +259,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
   const uint32_t tmem = ctl.tmem_base;
   const WorkerPlan plan = ctl.plan;
 
-  if (kSparse && warp == kProducerWarp) {
-    // ------------------------------------------------------------------ copy producer (sparse)
-    // Lanes map the 64 listed positions of a tile to cache rows (two each; -1 = no row). Each
-    // cache row is then copied by the whole warp with 16-byte cp.async copies into the same
-    // swizzled stage layout the TMA path writes: lane l takes unit l of the row's 512-byte
-    // latent slice (one row per warp instruction), and one 16-byte unit of eight rows' 64-byte
-    // RoPE slices. Every lane's copies of a tile complete one arrival on the stage barrier;
-    // rows that are not there are zero-filled without a read.
+  if (kSparse && (warp == kProducerWarp || warp == kConvWarp0)) {
+    // ------------------------------------------------------------------ copy producers (sparse)
+    // Two warps on different SM sub-partitions; warp 8 also loads the query. Warp h takes
+    // rows [32 h, 32 h + 32) of every tile: its lanes map those listed positions to cache
+    // rows (-1 = no row), then the whole warp copies each row with 16-byte cp.async copies
+    // into the same swizzled stage layout the TMA path writes: lane l takes unit l of the
+    // row's 512-byte latent slice (one row per warp instruction), and one 16-byte unit of
+    // four rows' 64-byte RoPE slices. Every lane's copies of a tile complete one arrival on
+    // the stage barrier; rows that are not there are zero-filled without a read.
+    const int half = warp == kProducerWarp ? 0 : 1;
     SegmentIter it(plan, a.seq_lens, a.B, a.bs, cap, w, a.status);
     Segment sg;
     uint32_t g = 0, seg = 0;
@@ -277,7 +279,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
     const uint32_t lat_dst = (lane >> 3) * kKvLatChunk;               // 64-channel chunk of the unit
     const uint32_t rope_src = 2 * kR + 64 * rank + 16 * (lane & 3);
     while (ok && it.next(sg)) {
-      if (lane == 0) {
+      if (half == 0 && lane == 0) {
         ok = mbar_wait<false>(smem_u32(&ctl.q_empty), (seg & 1) ^ 1, abort, timeout_ns);
         if (ok) {
           const uint32_t qbar = smem_u32(&ctl.q_full);
@@ -288,40 +290,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       for (int tile = sg.tile_begin; tile < sg.tile_end; ++tile, ++g) {
-        int rw[2];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int j = tile * kBS + 32 * hh + lane;   // list entry
-          int row = -1;
+        int rw = -1;
+        {
+          const int j = tile * kBS + 32 * half + lane;   // list entry
           if (j < sg.Lc) {
             const int t = __ldg(a.sel_idx + (size_t)sg.b * a.top_k + j);
             const int blk = (t >= 0 && t < a.max_blocks * kBS) ? __ldg(a.block_table + (size_t)sg.b * a.max_blocks + t / kBS) : -1;
             if (blk >= 0 && blk < a.num_blocks)
-              row = blk * kBS + t % kBS;
+              rw = blk * kBS + t % kBS;
             else
               set_status(a.status, MLA_ERR_BAD_BLOCK_ID);
           }
-          rw[hh] = row;
         }
         const uint32_t st = g % kStages, ph = (g / kStages) & 1;
         if (lane == 0) ok = mbar_wait<false>(smem_u32(&ctl.kv_empty[st]), ph ^ 1, abort, timeout_ns);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         const uint32_t base = sKv + st * kStageBytes;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll 8
-          for (int ii = 0; ii < 32; ++ii) {
-            const int i = 32 * hh + ii;
-            const int row = __shfl_sync(0xffffffffu, rw[hh], ii);
-            const char* src = cache + (size_t)(row < 0 ? 0 : row) * kRowBytes + lat_src;
-            cp_async_16(base + lat_dst + i * 128 + (((lane & 7) ^ (i & 7)) << 4), src, row < 0 ? 0u : 16u);
-          }
+        for (int ii = 0; ii < 32; ++ii) {
+          const int i = 32 * half + ii;
+          const int row = __shfl_sync(0xffffffffu, rw, ii);
+          const char* src = cache + (size_t)(row < 0 ? 0 : row) * kRowBytes + lat_src;
+          cp_async_16(base + lat_dst + i * 128 + (((lane & 7) ^ (i & 7)) << 4), src, row < 0 ? 0u : 16u);
         }
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int i = 8 * k + (lane >> 2);                 // rows 8k .. 8k + 7, four lanes each
-          const int row = __shfl_sync(0xffffffffu, rw[k >> 2], i & 31);
+        for (int k = 0; k < 4; ++k) {
+          const int ii = 8 * k + (lane >> 2);                // rows 8k .. 8k + 7 of the half, four lanes each
+          const int i = 32 * half + ii;
+          const int row = __shfl_sync(0xffffffffu, rw, ii);
           const char* src = cache + (size_t)(row < 0 ? 0 : row) * kRowBytes + rope_src;
           cp_async_16(base + 4 * kKvLatChunk + i * 64 + (((lane & 3) ^ ((i >> 1) & 3)) << 4), src, row < 0 ? 0u : 16u);
         }
@@ -332,7 +329,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8>(),
     cp_async_wait_all();
     if (lane == 0) {
       int dummy = 0;
-      for (uint32_t i = 0; i < kStages && i < g; ++i) {
+      for (uint32_t i = 0; half == 0 && i < kStages && i < g; ++i) {
         const uint32_t gl = g - 1 - i;
         mbar_wait<false>(smem_u32(&ctl.kv_full[gl % kStages]), (gl / kStages) & 1, &dummy, drain_ns);
       }
@@ -1072,13 +1069,13 @@ cudaError_t launch_tc_decode(const DecodeArgs& a, cudaStream_t s) {
   const uint64_t timeout_ns = wait_timeout_ns(), drain_ns = drain_timeout_ns();
   const dim3 grid(2 * a.W * n_rg);
   if (variant == 1)
-    tc_decode_kernel<true, false><<<grid, threads_for<true>(), Geo<true>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a, n_rg,
+    tc_decode_kernel<true, false><<<grid, threads_for<true, false>(), Geo<true>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a, n_rg,
                                                                                            timeout_ns, drain_ns);
   else if (variant == 2)
-    tc_decode_kernel<false, true><<<grid, threads_for<false>(), Geo<false>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a,
+    tc_decode_kernel<false, true><<<grid, threads_for<false, true>(), Geo<false>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a,
                                                                                              n_rg, timeout_ns, drain_ns);
   else
-    tc_decode_kernel<false, false><<<grid, threads_for<false>(), Geo<false>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a,
+    tc_decode_kernel<false, false><<<grid, threads_for<false, false>(), Geo<false>::kSmemBytes, s>>>(tqr, tkv, tkr, tsc, a,
                                                                                               n_rg, timeout_ns, drain_ns);
   return cudaGetLastError();
 }
