@@ -45,16 +45,19 @@
 //    the row sum over the unscaled p_t.
 //  * Warp roles: warps 0-3 own-lane softmax and epilogue, warps 4-7 peer-lane exchange
 //    and epilogue, warp 8 TMA producer, warp 9 TMEM allocator and single-thread MMA
-//    issuer, warps 10-11 FP8 converters; mbarrier pipelines between them. Every wait is
-//    bounded (timeout -> MLA_ERR_TIMEOUT, clean exit).
+//    issuer, warps 10-11 FP8 converters (sparse decode: warp 10 is a second copy warp);
+//    mbarrier pipelines between them. Every wait is bounded (timeout -> MLA_ERR_TIMEOUT,
+//    clean exit).
 //  * Sparse decode (DeepSeek Sparse Attention: "TransMLA & Sparse Latent Attention"
 //    lesson, Chapter 7 "DSA runs in MLA's MQA mode"): the same kernel over each
 //    sequence's list of selected positions instead of its whole length. The per-sequence
-//    length is the list's count, and tile t holds list entries [64 t, 64 t + 64); the
-//    producer warp maps them through the block table and copies the 64 token rows of
-//    the CTA's channel slice with 16-byte cp.async copies (one 512-byte row slice per warp
-//    instruction) into the same swizzled stage layout; each lane's copies complete one
-//    arrival on the stage barrier. Entries past the count are zero-filled without a read.
+//    length is the list's count, and tile t holds list entries [64 t, 64 t + 64). Two
+//    copy warps (8 and 10, on different SM sub-partitions, 32 rows each) map them through
+//    the block table and copy the token rows of the CTA's channel slice with 16-byte
+//    cp.async copies (one 512-byte row slice per warp instruction) into the same swizzled
+//    stage layout; each lane's copies complete one arrival on the stage barrier. Entries
+//    past the count are zero-filled without a read. The copies go through the LSU rather
+//    than TMA row gathers (four rows per load), which measured slower on B200.
 // The work split over workers (CTA pairs) is the flat block list plan of mla_device.cuh.
 #include <cuda.h>
 #include <cuda_fp16.h>
