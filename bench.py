@@ -88,7 +88,7 @@ KERNEL_SOURCES = {
 # The same for the sparse step's indexer (dram bytes per context token, batch 8 of the
 # 128K workload), keyed by the sources of mla_dsa.cu and its headers.
 DSA_TRAFFIC = {
-    "af77376c40dcd323": {"dsa_v32": (138.621952e6 + 4.314624e6) / (8 * 131072)},
+    "9f69c58ab496e496": {"dsa_v32": (138.620416e6 + 4.136448e6) / (8 * 131072)},
 }
 DSA_SOURCES = ("mla_dsa.cu", "ptx_sm100.cuh", "mla_device.cuh", "mla_internal.h")
 
