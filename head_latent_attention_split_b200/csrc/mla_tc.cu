@@ -329,15 +329,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for<kFp8, kS
       }
       ++seg;
     }
+    // Each lane waits for its own copies, so nothing lands after the CTA exits. (A stage
+    // barrier is no drain signal here: after a timeout one copy warp may have arrived on it
+    // and the other not.)
     cp_async_wait_all();
-    if (lane == 0) {
-      int dummy = 0;
-      for (uint32_t i = 0; half == 0 && i < kStages && i < g; ++i) {
-        const uint32_t gl = g - 1 - i;
-        mbar_wait<false>(smem_u32(&ctl.kv_full[gl % kStages]), (gl / kStages) & 1, &dummy, drain_ns);
-      }
-      if (!ok) set_status(a.status, MLA_ERR_TIMEOUT);
-    }
+    if (lane == 0 && !ok) set_status(a.status, MLA_ERR_TIMEOUT);
   } else if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {

@@ -252,6 +252,49 @@ def test_sparse_decode_random_lists_and_edges(small, kernel):
 
 
 @pytest.mark.parametrize("kernel", SPARSE_KERNELS)
+def test_sparse_decode_wait_timeout_expires_cleanly(small, kernel):
+    """A pipeline wait limit far below a tile's time makes the sparse decode's waits run out
+    (both copy warps and the consumers): the call returns, the status reads MLA_ERR_TIMEOUT
+    once, every row is NaN throughout or right, and the next call at the default limit
+    matches the oracle."""
+    torch = _torch()
+    mla = _mla()
+    inp = small
+    rng = np.random.default_rng(5)
+    k = 512
+    lens = inp["seq_lens"]
+    cnt = np.minimum(lens, k).astype(np.int32)
+    idx = np.full((3, k), -1, np.int32)
+    for b in range(3):
+        idx[b, :cnt[b]] = rng.choice(int(lens[b]), size=int(cnt[b]), replace=False)
+    ro, rl = oracle_sparse(inp, idx, cnt)
+    w = inp["workload"]
+    t = W.to_torch(inp)
+    assert mla.wait_timeout_ns() == 2_000_000_000
+    mla.set_wait_timeout_ns(200)
+    try:
+        out, lse = mla.sparse_decode(t["q_lat"], t["q_rope"], t["kv_cache"], t["block_table"], _dev(idx),
+                                     _dev(cnt), w.scale, kernel=kernel)
+        torch.cuda.synchronize()
+    finally:
+        mla.set_wait_timeout_ns(0)
+    assert mla.wait_timeout_ns() == 2_000_000_000
+    assert mla.device_status() == 8           # MLA_ERR_TIMEOUT
+    assert mla.device_status() == 0
+    o = out.double().cpu().numpy()
+    l = lse.double().cpu().numpy()
+    assert np.isnan(l).any()
+    for b in range(w.B):
+        for h in range(w.H):
+            if np.isnan(l[b, 0, h]):
+                assert np.isnan(o[b, 0, h]).all()
+            else:
+                assert abs(l[b, 0, h] - rl[b, 0, h]) <= LSE_TOL
+    out2, lse2 = gpu_sparse(inp, idx, cnt, kernel)
+    compare(out2, lse2, ro, rl, TOL[W.BF16], "sparse decode after the timeout")
+
+
+@pytest.mark.parametrize("kernel", SPARSE_KERNELS)
 def test_sparse_decode_every_token_is_dense(small, kernel):
     # a list holding every position equals the dense decode (the oracle's dense decode)
     inp = small
