@@ -295,6 +295,114 @@ mla_status_t host_io_layout(const mla_decode_params_t* p, HostIoLayout* H) {
 }
 }  // namespace
 
+namespace {
+// Sequence chunks of a host-I/O step. With several chunks, the copies of one chunk overlap the
+// decode of another: host->device copies on one internal stream, the decodes on the caller's
+// stream, device->host copies on a second internal stream. One chunk for small steps, where
+// the extra launches would cost more than the copies they hide.
+constexpr int kHostIoChunks = 4;
+constexpr size_t kHostIoChunkMinBytes = size_t(8) << 20;
+constexpr int kHostIoChunkMinBatch = 16;
+
+int host_io_chunk_count(const mla_decode_params_t* p, const HostIoLayout& H) {
+  const size_t io = H.q_bytes + H.qr_bytes + H.out_bytes + H.lse_bytes;
+  return (p->batch >= kHostIoChunkMinBatch && io >= kHostIoChunkMinBytes) ? kHostIoChunks : 1;
+}
+
+// Per host thread and device, so the copy streams of one thread's calls stay in call order.
+struct CopyStreams {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+};
+CopyStreams* copy_streams(int dev) {
+  thread_local CopyStreams S[64];
+  if (dev < 0 || dev >= 64) return nullptr;
+  CopyStreams& c = S[dev];
+  if (!c.h2d && cudaStreamCreateWithFlags(&c.h2d, cudaStreamNonBlocking) != cudaSuccess) c.h2d = nullptr;
+  if (!c.d2h && cudaStreamCreateWithFlags(&c.d2h, cudaStreamNonBlocking) != cudaSuccess) c.d2h = nullptr;
+  return (c.h2d && c.d2h) ? &c : nullptr;
+}
+
+struct HostIoArgs {
+  const void *q_lat, *q_rope, *kv_cache, *k_rope_cache;
+  const float* kv_scale;
+  const int32_t *block_table, *seq_lens;
+  void* out;
+  float* lse;
+};
+
+// The chunked step. Sets *ran to false, with nothing enqueued, when a chunk's staging pointers
+// would break the decode's 16-byte alignment (the caller then runs the step as one chunk).
+mla_status_t host_io_chunked(const mla_decode_params_t* p, const HostIoLayout& H, int K, const HostIoArgs& h,
+                             char* ws, cudaStream_t s, bool* ran) {
+  *ran = false;
+  const int B = p->batch;
+  const int nb = ((B + K - 1) / K + 3) / 4 * 4;   // sequences per chunk, a multiple of 4
+  const size_t q1 = H.q_bytes / B, qr1 = H.qr_bytes / B, bt1 = H.bt_bytes / B, out1 = H.out_bytes / B,
+               lse1 = H.lse_bytes / B;
+  for (int b0 = 0; b0 < B; b0 += nb) {
+    const size_t offs[] = {H.q_off + b0 * q1,     H.qr_off + b0 * qr1,   H.bt_off + b0 * bt1,
+                           H.sl_off + b0 * size_t(4), H.out_off + b0 * out1, H.lse_off + b0 * lse1};
+    for (size_t o : offs)
+      if (o % 16) return MLA_OK;
+  }
+  CopyStreams* cs = copy_streams(current_device());
+  if (!cs) return MLA_ERR_CUDA;
+  cudaEvent_t ev[2 * kHostIoChunks + 2] = {};
+  int nev = 0;
+  auto event = [&]() -> cudaEvent_t {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    ev[nev++] = e;
+    return e;
+  };
+  mla_status_t st = MLA_OK;
+  *ran = true;
+  do {
+    cudaEvent_t start = event();
+    if (!start || cudaEventRecord(start, s) != cudaSuccess || cudaStreamWaitEvent(cs->h2d, start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(cs->d2h, start, 0) != cudaSuccess) {
+      st = MLA_ERR_CUDA;
+      break;
+    }
+    for (int b0 = 0; b0 < B && st == MLA_OK; b0 += nb) {
+      const int n = B - b0 < nb ? B - b0 : nb;
+      struct Copy { void* dst; const void* src; size_t n; };
+      const Copy h2d[] = {{ws + H.q_off + b0 * q1, (const char*)h.q_lat + b0 * q1, n * q1},
+                          {ws + H.qr_off + b0 * qr1, (const char*)h.q_rope + b0 * qr1, n * qr1},
+                          {ws + H.bt_off + b0 * bt1, (const char*)h.block_table + b0 * bt1, n * bt1},
+                          {ws + H.sl_off + b0 * size_t(4), (const char*)h.seq_lens + b0 * size_t(4), n * size_t(4)}};
+      for (const Copy& c : h2d)
+        if (c.n && cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, cs->h2d) != cudaSuccess) st = MLA_ERR_CUDA;
+      cudaEvent_t in = event(), done = event();
+      if (st || !in || !done || cudaEventRecord(in, cs->h2d) != cudaSuccess || cudaStreamWaitEvent(s, in, 0) != cudaSuccess) {
+        st = MLA_ERR_CUDA;
+        break;
+      }
+      mla_decode_params_t pc = *p;
+      pc.batch = n;
+      st = mla_decode(&pc, ws + H.q_off + b0 * q1, p->rope_dim ? ws + H.qr_off + b0 * qr1 : nullptr, h.kv_cache,
+                      h.k_rope_cache, h.kv_scale, (const int32_t*)(ws + H.bt_off + b0 * bt1),
+                      (const int32_t*)(ws + H.sl_off + b0 * size_t(4)), ws + H.out_off + b0 * out1,
+                      (float*)(ws + H.lse_off + b0 * lse1), ws + H.ws_off, H.ws_bytes, s);
+      if (st) break;
+      if (cudaEventRecord(done, s) != cudaSuccess || cudaStreamWaitEvent(cs->d2h, done, 0) != cudaSuccess ||
+          cudaMemcpyAsync((char*)h.out + b0 * out1, ws + H.out_off + b0 * out1, n * out1, cudaMemcpyDeviceToHost,
+                          cs->d2h) != cudaSuccess ||
+          cudaMemcpyAsync((char*)h.lse + b0 * lse1, ws + H.lse_off + b0 * lse1, n * lse1, cudaMemcpyDeviceToHost,
+                          cs->d2h) != cudaSuccess)
+        st = MLA_ERR_CUDA;
+    }
+    if (st) break;
+    // the caller's stream covers the whole step, the last copy back included
+    cudaEvent_t end = event();
+    if (!end || cudaEventRecord(end, cs->d2h) != cudaSuccess || cudaStreamWaitEvent(s, end, 0) != cudaSuccess)
+      st = MLA_ERR_CUDA;
+  } while (false);
+  for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);   // released once the work that uses them is done
+  return st;
+}
+}  // namespace
+
 mla_status_t mla_decode_host_io_workspace_size(const mla_decode_params_t* p, size_t* bytes) {
   if (!bytes) return MLA_ERR_INVALID_ARG;
   HostIoLayout H;
@@ -319,6 +427,14 @@ mla_status_t mla_decode_host_io(const mla_decode_params_t* p, const void* q_lat_
   if (!aligned(workspace, 256)) return MLA_ERR_ALIGNMENT;
   char* ws = (char*)workspace;
   cudaStream_t s = (cudaStream_t)stream;
+  const int K = host_io_chunk_count(p, H);
+  if (K > 1) {
+    const HostIoArgs h{q_lat_host, q_rope_host, kv_cache, k_rope_cache, kv_scale, block_table_host, seq_lens_host,
+                       out_host, lse_host};
+    bool ran = false;
+    st = host_io_chunked(p, H, K, h, ws, s, &ran);
+    if (ran || st) return st;
+  }
   struct Copy { void* dst; const void* src; size_t n; };
   const Copy h2d[] = {{ws + H.q_off, q_lat_host, H.q_bytes},
                       {ws + H.qr_off, q_rope_host, H.qr_bytes},

@@ -149,9 +149,17 @@ mla_status_t mla_decode_host_io_workspace_size(const mla_decode_params_t* params
 
 /* One decode step whose per-step tensors are in HOST memory (pinned memory makes the
  * copies asynchronous): q_lat, q_rope, block_table, seq_lens are copied to the
- * device, the step runs, out and lse are copied back, all on `stream`. The cache
- * (kv_cache, k_rope_cache, kv_scale) stays device-resident. The call returns once
- * the work is enqueued; synchronise the stream before reading out / lse. */
+ * device, the step runs, out and lse are copied back. The cache (kv_cache,
+ * k_rope_cache, kv_scale) stays device-resident. The call returns once the work is
+ * enqueued; synchronise `stream` before reading out / lse (the stream's work covers the
+ * whole step, the copies back included).
+ * A step of at least 16 sequences whose per-step copies (q_lat, q_rope, out, lse) reach
+ * 8 MiB runs as four chunks of consecutive sequences (a multiple of 4 each): the copies
+ * of one chunk overlap the decode of another, on two copy streams the library keeps per
+ * host thread and device, ordered against `stream` by events. Each chunk is a decode of
+ * its own (its own split of the sequences over the workers), so such a step can differ
+ * from one mla_decode over the whole batch in the last bits, within the decode's
+ * accuracy; smaller steps run as one chunk on `stream` and match mla_decode exactly. */
 mla_status_t mla_decode_host_io(const mla_decode_params_t* params, const void* q_lat_host,
                                 const void* q_rope_host, const void* kv_cache,
                                 const void* k_rope_cache, const float* kv_scale,

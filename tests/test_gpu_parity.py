@@ -267,6 +267,37 @@ def test_host_io_matches_device_call(mla, small_cases, kernel):
     assert np.array_equal(o_h.double().numpy(), o_d) and np.array_equal(l_h.double().numpy(), l_d)
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_host_io_chunked_pipeline(mla, kernel):
+    """A host-I/O step large enough to be pipelined (B = 32, 128 heads: 8.5 MiB of per-step
+    copies) runs as four chunks of 8 consecutive sequences whose copies overlap the other
+    chunks' decodes. Each chunk is its own decode: the result equals, bit for bit, the device
+    decode of each 8-sequence slice, and matches the oracle."""
+    import torch
+    rng = np.random.default_rng(21)
+    wl = W.WORKLOADS[2].with_(B=32, seq_lens=tuple(int(x) for x in rng.integers(1, 700, 32)))
+    inp = W.make_inputs(wl)
+    if not kernel_ok(mla, inp, kernel):
+        pytest.skip(kernel)
+    ref_o, ref_l = oracle.decode_inputs(inp)
+    t = W.to_torch(inp)
+    pin = lambda x: x.cpu().pin_memory()  # noqa: E731
+    o_h, l_h = mla.decode_host_io(pin(t["q_lat"]), pin(t["q_rope"]), t["kv_cache"], pin(t["block_table"]),
+                                  pin(t["seq_lens"]), wl.scale, wl.causal, kernel=kernel)
+    torch.cuda.synchronize()
+    assert mla.device_status() == 0
+    o_h, l_h = o_h.double().numpy(), l_h.double().numpy()
+    compare(o_h, l_h, ref_o, ref_l, TOL[wl.cache_dtype], f"chunked host I/O ({kernel})")
+    for b0 in range(0, 32, 8):
+        sl = slice(b0, b0 + 8)
+        o_d, l_d = mla.decode(t["q_lat"][sl].contiguous(), t["q_rope"][sl].contiguous(), t["kv_cache"],
+                              t["block_table"][sl].contiguous(), t["seq_lens"][sl].contiguous(), wl.scale,
+                              wl.causal, kernel=kernel)
+        torch.cuda.synchronize()
+        assert np.array_equal(o_h[sl], o_d.double().cpu().numpy()), f"chunk {b0}"
+        assert np.array_equal(l_h[sl], l_d.double().cpu().numpy()), f"chunk {b0}"
+
+
 # ---------------------------------------------------------------------------- full-size workloads
 _FULL = {}
 
