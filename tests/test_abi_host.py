@@ -116,6 +116,38 @@ def test_batch_zero_is_a_noop(m):
     assert _call(m, p, q_lat=None, kv_cache=None) == 0
 
 
+def _host_io(m, p, **ptrs):
+    from head_latent_attention_split_b200 import binding
+    args = dict(q_lat_host=FAKE, q_rope_host=FAKE, kv_cache=FAKE, k_rope_cache=None, kv_scale=None,
+                block_table_host=FAKE, seq_lens_host=FAKE, out_host=FAKE, lse_host=FAKE, workspace=FAKE,
+                workspace_bytes=1 << 30)
+    args.update(ptrs)
+    return binding.mla_decode_host_io(p, stream=0, check=False, **args)
+
+
+def test_host_io_workspace_size_formula(m):
+    # device staging of q_lat, q_rope, block_table, seq_lens, out, lse after mla_decode's own
+    # workspace, each region 256-byte aligned (f32 queries and output here)
+    B, Sq, H, r, d_r, mb = 5, 2, 8, 32, 8, 3
+    p = _p(m, B=B, Sq=Sq, H=H, r=r, d_r=d_r, max_blocks_per_seq=mb, num_blocks=16, num_workers=7)
+    rows = B * Sq * H
+    al = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    want = (al(m.workspace_size(p)) + al(rows * r * 4) + al(rows * d_r * 4) + al(B * mb * 4) + al(B * 4)
+            + al(rows * r * 4) + al(rows * 4))
+    assert m.host_io_workspace_size(p) == want
+
+
+def test_host_io_rejects_bad_arguments_on_host(m):
+    p = _p(m)
+    need = m.host_io_workspace_size(p)
+    for k in ("q_lat_host", "q_rope_host", "block_table_host", "seq_lens_host", "out_host", "lse_host", "workspace"):
+        assert _host_io(m, p, **{k: None}) == 1, k                  # MLA_ERR_INVALID_ARG
+    assert _host_io(m, p, workspace_bytes=need - 1) == 4            # MLA_ERR_WORKSPACE_TOO_SMALL
+    assert _host_io(m, p, workspace=FAKE + 16, workspace_bytes=need) == 3   # MLA_ERR_ALIGNMENT
+    assert _host_io(m, _p(m, Sq=0)) == 1                            # bad params, nothing enqueued
+    assert _host_io(m, _p(m, B=0), q_lat_host=None, workspace=None) == 0   # empty batch: a no-op
+
+
 def test_workspace_size_formula(m):
     p = _p(m, B=5, Sq=2, H=8, r=32, num_workers=7)
     rows, slots = 2 * 8, 7 + 5 - 1
